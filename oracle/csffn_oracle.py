@@ -1,0 +1,277 @@
+"""CPU oracle for the contextually sparse gated FFN at decode time.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import or call
+this module: only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` do.  It shares
+no code with the CUDA library.
+
+Every function computes the plain definition in float64 with numpy (matrix
+products are the only library primitive used), on exactly the operand bits
+the GPU receives (bf16 bit patterns as uint16, or float32).  No blocking,
+fusion or reordering: the sparse method reaches the same result faster.
+
+Sources (page titles; sections, figures and tables on each):
+  [CATS]   "CATS: Contextually-Aware Thresholding for Sparsity in Large
+           Language Models", abstract: a new non-linear activation that
+           thresholds the gate activations; a custom GPU kernel whose entry
+           points fuse the gate GEMV with the compare and a flag-gated GEMV.
+  [SVDP]   "SVD Contextual Sparsity Predictors for Fast LLM Inference",
+           abstract; Fig. 1 (offline SVD predictors with calibrated per-neuron
+           thresholds, run ahead of each FFN block); Fig. 2 (zero threshold
+           gives false negatives); Fig. 3 (gate then up run sequentially on the
+           predicted-active neurons, ReGLU); Table 3 ("+ Bias calibration").
+  [SIRIUS] "Sirius: Contextual Sparsity with Correction for Efficient LLMs",
+           abstract, and its summary page, section "Approach": the sparse and
+           the full model share weights; the full model verifies a chunk of
+           sparse-generated tokens in parallel.
+
+Readings taken where the pages are silent (each one is listed in the design
+notes): the CATS threshold applies to the gate output SiLU(z) with strict
+``|a| > t``; the quantile is the lower order statistic v_(ceil(s*M)) without
+interpolation; t is one scalar per layer pooled over neurons x calibration
+vectors; the SVD predictor factors W_gate^T = U S V^T as U_r = U[:, :r] S_r
+(stored transposed, [r, d]) and V_r = V[:, :r] ([h, r]); tau_i is the
+per-neuron lower order statistic of the predictor output at q; the gate bias
+is an explicit additive vector; RMSNorm has unit gain and eps = 1e-6.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+RMS_EPS = 1e-6
+
+
+def decode(a) -> np.ndarray:
+    """Exact float64 value of a stored operand: bf16 bit patterns (uint16) or float32."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z) = z / (1 + e^{-z}) (the SwiGLU gate activation)."""
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def relu(z: np.ndarray) -> np.ndarray:
+    """ReLU(z) = max(z, 0) (the ReGLU gate activation of [SVDP])."""
+    return np.maximum(z, 0.0)
+
+
+def activation(z: np.ndarray, act: str) -> np.ndarray:
+    if act == "silu":
+        return silu(z)
+    if act == "relu":
+        return relu(z)
+    raise ValueError(act)
+
+
+def _tokens(x) -> np.ndarray:
+    x = decode(x)
+    return x[None, :] if x.ndim == 1 else x
+
+
+def gate_preactivation(x, layer) -> np.ndarray:
+    """z[b, i] = x_b . W_gate[i, :] + beta_i  ->  [B, h]."""
+    z = _tokens(x) @ decode(layer.w_gate).T
+    if layer.bias is not None:
+        z = z + decode(layer.bias)[None, :]
+    return z
+
+
+def gate_activation(x, layer) -> np.ndarray:
+    """a = act(z): SiLU for SwiGLU, ReLU for ReGLU  ->  [B, h]."""
+    return activation(gate_preactivation(x, layer), layer.act)
+
+
+def up_projection(x, layer) -> np.ndarray:
+    """u[b, i] = x_b . W_up[i, :]  ->  [B, h]."""
+    return _tokens(x) @ decode(layer.w_up).T
+
+
+def down_projection(g: np.ndarray, layer) -> np.ndarray:
+    """out[b, :] = sum_i g[b, i] * W_down^T[i, :]  ->  [B, d]."""
+    return g @ decode(layer.w_down_t)
+
+
+def dense_ffn(x, layer) -> np.ndarray:
+    """Dense gated FFN: out = (act(x W_gate^T + beta) * (x W_up^T)) W_down.
+
+    This is the full model's FFN that verifies a chunk of sparse tokens
+    ([SIRIUS] "Approach": sparse and full model share the weights).
+    """
+    return down_projection(gate_activation(x, layer) * up_projection(x, layer), layer)
+
+
+def cats_mask(a: np.ndarray, t: float) -> np.ndarray:
+    """[CATS] thresholding: neuron i is active for token b iff |a[b, i]| > t (strict)."""
+    return np.abs(a) > t
+
+
+def sparse_ffn(x, layer, mask: np.ndarray) -> np.ndarray:
+    """The dense FFN evaluated with the activations outside ``mask`` set to zero.
+
+    ``mask`` is [B, h] (or [h], broadcast over tokens).  This is the result the
+    sparse executor must reach by reading only the active rows.
+    """
+    a = gate_activation(x, layer)
+    m = np.asarray(mask, dtype=bool)
+    if m.ndim == 1:
+        m = np.broadcast_to(m[None, :], a.shape)
+    return down_projection(np.where(m, a, 0.0) * up_projection(x, layer), layer)
+
+
+def cats_ffn(x, layer, t: float) -> tuple:
+    """[CATS] sparse FFN at threshold t -> (out [B, d], per-token mask [B, h])."""
+    m = cats_mask(gate_activation(x, layer), t)
+    return sparse_ffn(x, layer, m), m
+
+
+def union_mask(mask: np.ndarray) -> np.ndarray:
+    """Rows a small batch must read: the union over tokens of the per-token masks -> [h]."""
+    return np.asarray(mask, dtype=bool).reshape(-1, np.shape(mask)[-1]).any(axis=0)
+
+
+def active_indices(row_mask: np.ndarray) -> np.ndarray:
+    """Ascending int32 indices of the set entries of a [h] mask."""
+    return np.flatnonzero(np.asarray(row_mask, dtype=bool)).astype(np.int32)
+
+
+def order_statistic_rank(s: float, m: int) -> int:
+    """k = ceil(s * m), clamped to [0, m].
+
+    s is first taken at float32 precision (the type the library interface
+    carries), then the product is evaluated exactly; 0.9 of 50 values is 45.
+    """
+    k = math.ceil(Fraction(float(np.float32(s))) * m)
+    return min(max(k, 0), m)
+
+
+def calibrate_global(x_cal, layer, s: float) -> float:
+    """One CATS threshold per layer: the s-quantile of |a| pooled over calibration set x neurons.
+
+    M = N*h values |a|, sorted ascending; k = ceil(s*M); t = v_(k) (1-indexed),
+    t = 0 when k = 0.  On the calibration set #{|a| <= t} >= k, with equality
+    when no ties occur.
+    """
+    v = np.sort(np.abs(gate_activation(x_cal, layer)).ravel())
+    k = order_statistic_rank(s, v.size)
+    return 0.0 if k == 0 else float(v[k - 1])
+
+
+def kth_smallest(values: np.ndarray, k: int) -> float:
+    """v_(k) of a flat array (1-indexed); used for checking order-statistic selection."""
+    v = np.sort(np.asarray(values, dtype=np.float64).ravel())
+    return float(v[k - 1])
+
+
+def svd_factors(w_gate, r: int) -> tuple:
+    """[SVDP] abstract / Fig. 1: rank-r truncated SVD of the gate projection.
+
+    The gate maps a row vector x to x W_gate^T, so the projection matrix is
+    W_gate^T (d x h) = U S V^T.  Returns (U_r^T [r, d] = (U[:, :r] S_r)^T,
+    V_r [h, r] = V[:, :r]) in float64; x U_r V_r^T approximates x W_gate^T.
+    """
+    u, s, vt = np.linalg.svd(decode(w_gate).T, full_matrices=False)
+    return (u[:, :r] * s[None, :r]).T.copy(), vt[:r, :].T.copy()
+
+
+def predict(x, u_rt, v_r, bias=None) -> np.ndarray:
+    """[SVDP] Fig. 1: predictor output p = (x U_r) V_r^T + beta  ->  [B, h]."""
+    p = (_tokens(x) @ decode(u_rt).T) @ decode(v_r).T
+    if bias is not None:
+        p = p + decode(bias)[None, :]
+    return p
+
+
+def calibrate_per_neuron(x_cal, u_rt, v_r, bias, q: float) -> np.ndarray:
+    """[SVDP] Fig. 1 / Table 3 "bias calibration": per-neuron thresholds tau [h].
+
+    tau_i = k-th smallest of {p_i(x_n)} over the N calibration vectors,
+    k = ceil(q*N); tau_i = -inf when k = 0.  Neuron i is then predicted active
+    on at most a (1-q) fraction of the calibration inputs.
+    """
+    p = np.sort(predict(x_cal, u_rt, v_r, bias), axis=0)
+    k = order_statistic_rank(q, p.shape[0])
+    if k == 0:
+        return np.full(p.shape[1], -np.inf)
+    return p[k - 1, :].copy()
+
+
+def predicted_mask(p: np.ndarray, tau: np.ndarray) -> np.ndarray:
+    """P = {i : p_i > tau_i} per token -> [B, h]."""
+    return p > np.asarray(tau, dtype=np.float64)[None, :]
+
+
+def reglu_sequential(x, layer, pred_mask: np.ndarray) -> tuple:
+    """[SVDP] Fig. 3: gate on the predicted set P, then up/down only on A = {i in P : z_i > 0}.
+
+    Returns (out [B, d], A [B, h]).  ``pred_mask`` is per token [B, h] or [h].
+    """
+    z = gate_preactivation(x, layer)
+    p = np.asarray(pred_mask, dtype=bool)
+    if p.ndim == 1:
+        p = np.broadcast_to(p[None, :], z.shape)
+    a_mask = p & (z > 0.0)
+    out = down_projection(np.where(a_mask, z, 0.0) * up_projection(x, layer), layer)
+    return out, a_mask
+
+
+def rmsnorm(v: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
+    """RMSNorm with unit gain: v / sqrt(mean(v^2) + eps), per row."""
+    v = np.asarray(v, dtype=np.float64)
+    return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+
+
+def round_to_bf16(v: np.ndarray) -> np.ndarray:
+    """Value of v after rounding to bfloat16 (nearest, ties to even), as float64.
+
+    Done through PyTorch's CPU cast, independently of the input encoder.
+    """
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float64))
+    return t.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def stack_layer(h: np.ndarray, layer, t=None, mask=None) -> tuple:
+    """One residual block of the FFN stack: h + FFN(bf16(RMSNorm(h))).
+
+    With ``mask`` the FFN is the sparse one on that mask; with ``t`` the CATS
+    mask at t; with neither, the dense FFN.  Returns (h_next, xn, mask_used).
+    """
+    xn = round_to_bf16(rmsnorm(h))
+    if mask is None and t is not None:
+        mask = cats_mask(gate_activation(xn, layer), t)
+    y = dense_ffn(xn, layer) if mask is None else sparse_ffn(xn, layer, mask)
+    return np.asarray(h, dtype=np.float64) + y, xn, mask
+
+
+def sirius_round(x_steps, layer, t: float) -> tuple:
+    """[SIRIUS] "Approach", FFN part only: the sparse FFN drafts each of the chunk's
+    tokens one at a time, then the dense FFN verifies the whole chunk in one batch.
+
+    Returns (sparse outputs [T, d], dense outputs [T, d], masks [T, h]).
+    """
+    x = _tokens(x_steps)
+    sparse, masks = [], []
+    for b in range(x.shape[0]):
+        o, m = cats_ffn(x[b], layer, t)
+        sparse.append(o[0])
+        masks.append(m[0])
+    return np.stack(sparse), dense_ffn(x, layer), np.stack(masks)
+
+
+def rel_l2(y, y_ref) -> float:
+    """max over vectors of ||y - y_ref||_2 / ||y_ref||_2 (0/0 counts as 0)."""
+    y = np.atleast_2d(np.asarray(y, dtype=np.float64))
+    r = np.atleast_2d(np.asarray(y_ref, dtype=np.float64))
+    num = np.linalg.norm(y - r, axis=-1)
+    den = np.linalg.norm(r, axis=-1)
+    out = np.where(den > 0, num / np.where(den > 0, den, 1.0), np.where(num > 0, np.inf, 0.0))
+    return float(out.max()) if out.size else 0.0
