@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the contextually sparse FFN decode step on B200.
+
+Workload: LLaMA-2-7B-shaped SwiGLU FFN layer (d=4096, h=11008), bf16 weights, fp32
+accumulation, batch-1 decode, CATS threshold calibrated by csffn_calibrate_threshold
+on 512 seeded calibration vectors at 50% target sparsity (70% and 90% and the dense
+path of the same library are measured too and reported under "detail").
+
+A step is one CATS decode of one layer: csffn_gate_mask (gate GEMV + SiLU + threshold
++ compaction) then csffn_sparse_ffn_forward (gathered up and down projections).  The
+timed steps rotate over 8 distinct layer weight sets (2.2 GB, many times the 126 MB L2)
+so no step reads weights that an earlier step left in L2.  K steps are captured in one
+CUDA graph and timed with CUDA events on the capture stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csffn|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica (the decode step has no
+exchange step); the time is the max over ranks and ``value`` is the whole-job time
+per layer-step (max time / (N * K)).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+METRIC = "sparse-FFN decode µs/layer + achieved HBM GB/s vs 8 TB/s, speedup over dense"
+UNIT = "µs/layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+D, H = 4096, 11008
+N_ROT = 8
+N_TOKENS = 64
+PROFILE_SUMMARY = os.path.join(HERE, "profiles", "gate_mask_llama2_7b_b1.md")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["csffn", "reference"], default="csffn")
+    ap.add_argument("--sparsity", type=float, default=0.5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-detail", action="store_true", help="skip the 70%/90%/dense detail runs")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a float over ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_layer(t_max_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per layer-step: the slowest rank's time over all ranks' layer-steps."""
+    return t_max_ms * 1000.0 / (steps * world)
+
+
+# ---------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the measured window."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if self.bus_id:
+                cmd += ["-i", self.bus_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def pci_bus_id(torch, dev: int) -> str:
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return ""
+
+
+# ---------------------------------------------------------------------------------- peaks
+
+def measured_hbm_gbs():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(HERE, "contextual_sparsity_ffn_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram bytes per gate-kernel launch from the committed ncu summary, if it matches this source."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    hsh = re.search(r"csrc_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not hsh or hsh.group(1) != csrc_hash():
+        return None
+    return float(m.group(1))
+
+
+# ---------------------------------------------------------------------------------- csffn arm
+
+def build_workload(torch, cs, synth, sparsities):
+    """8 rotation layers on the device, their thresholds per sparsity, and seeded tokens."""
+    layers, thresholds = [], {s: [] for s in sparsities}
+    for li in range(N_ROT):
+        spec, _, xc = synth.llama2_7b_swiglu(li, n_eval=1, n_calib=512)
+        layer = cs.FFNLayer.from_spec(spec, "cuda")
+        xcal = cs.to_device(xc, "cuda")
+        for s in sparsities:
+            t = torch.zeros(1, device="cuda")
+            cs.calibrate_threshold(layer, xcal, s, 0, t)
+            thresholds[s].append(float(t.item()))
+        layers.append(layer)
+        del spec, xc, xcal
+    xs = synth.make_tokens(1, 0, synth.ROLE_EVAL, N_TOKENS, D, "bf16", rms_normalise=True)
+    return layers, thresholds, cs.to_device(xs, "cuda")
+
+
+def run_graph_steps(torch, step_fn, steps, warmup, stream, events_cb=None):
+    """Capture `steps` calls of step_fn(k) into one graph; replay warm-up, then time one replay."""
+    with torch.cuda.stream(stream):
+        for k in range(min(warmup, 3)):
+            step_fn(k)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for k in range(steps):
+            step_fn(k)
+    return g
+
+
+def csffn_arm(args, world, rank, local):
+    import torch
+    from contextual_sparsity_ffn_b200 import binding as cs
+    from contextual_sparsity_ffn_b200 import synth
+
+    torch.cuda.set_device(local)
+    dist = init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    sparsities = [args.sparsity] + ([] if args.no_detail else [s for s in (0.5, 0.7, 0.9) if s != args.sparsity])
+    layers, thr, xs = build_workload(torch, cs, synth, sparsities)
+    buf = cs.DecodeBuffers.new(layers[0], 1)
+    out = torch.zeros(1, D, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+    K, W = args.steps, args.warmup
+
+    def sparse_step(s, gate_events=None):
+        def f(k):
+            li = k % N_ROT
+            x = xs[k % N_TOKENS: k % N_TOKENS + 1]
+            if gate_events is not None:
+                gate_events[k][0].record()
+            cs.gate_mask(layers[li], x, thr[s][li], buf.idx, buf.count, buf.a_val, buf.ws)
+            if gate_events is not None:
+                gate_events[k][1].record()
+            cs.sparse_ffn_forward(layers[li], x, buf.idx, buf.count, buf.a_val, out, buf.ws)
+        return f
+
+    def dense_step(k):
+        li = k % N_ROT
+        cs.dense_ffn_forward(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], out, buf.ws)
+
+    def time_graph(g, replays_warm):
+        for _ in range(replays_warm):
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record()
+            g.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
+
+    # ---- main measurement: K steps at the headline sparsity, gate-kernel events inside the graph
+    try:
+        gate_ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K)]
+        g_main = run_graph_steps(torch, sparse_step(args.sparsity, gate_ev), K, W, stream)
+        gate_in_graph = True
+    except Exception:
+        gate_ev = None
+        torch.cuda.synchronize()
+        g_main = run_graph_steps(torch, sparse_step(args.sparsity), K, W, stream)
+        gate_in_graph = False
+    bus = pci_bus_id(torch, local)
+    sampler = ClockSampler(bus).start()
+    # warm-up: W steps' worth of replays plus a sustained second so clocks settle and are sampled
+    warm_replays = max(1, (W + K - 1) // K)
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        g_main.replay()
+        torch.cuda.synchronize()
+    ms = time_graph(g_main, warm_replays)
+    clocks = sampler.stop()
+    ms_max = max_over_ranks(ms, world, dev)
+    if gate_in_graph:
+        gate_ms = [a.elapsed_time(b) for a, b in gate_ev]
+    else:
+        gate_ms = time_gate_eager(torch, cs, layers, thr[args.sparsity], xs, buf, stream, K)
+    gate_avg_us = 1000.0 * float(np.mean(gate_ms))
+
+    # active rows actually read per step (deterministic; recomputed eagerly)
+    counts = []
+    for k in range(min(K, N_ROT * N_TOKENS)):
+        li = k % N_ROT
+        cs.gate_mask(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], thr[args.sparsity][li],
+                     buf.idx, buf.count, buf.a_val, buf.ws)
+        counts.append(int(buf.count.item()))
+    n_act = float(np.mean(counts))
+
+    def step_bytes(n_active):
+        # all of W_gate + gathered W_up and W_down^T rows + x, out, idx, a_val
+        return 2.0 * H * D + 2.0 * 2.0 * n_active * D + 2 * D + 4 * D + 8.0 * n_active
+
+    peak, peak_kind = measured_hbm_gbs()
+    us = whole_job_us_per_layer(ms_max, K, world)
+    us_gpu = ms_max * 1000.0 / K  # one GPU's time per layer-step
+    gbs = step_bytes(n_act) / (us_gpu * 1e-6) / 1e9  # per GPU
+    gate_bytes = 2.0 * H * D + 2 * D + 8.0 * n_act + 4.0 * n_act
+    gate_gbs = gate_bytes / (gate_avg_us * 1e-6) / 1e9
+
+    detail = {}
+    if not args.no_detail:
+        for s in sparsities[1:]:
+            g = run_graph_steps(torch, sparse_step(s), K, W, stream)
+            t = time_graph(g, warm_replays)
+            t = max_over_ranks(t, world, dev)
+            cnt = []
+            for k in range(min(K, N_ROT * N_TOKENS)):
+                li = k % N_ROT
+                cs.gate_mask(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], thr[s][li], buf.idx, buf.count,
+                             buf.a_val, buf.ws)
+                cnt.append(int(buf.count.item()))
+            u = whole_job_us_per_layer(t, K, world)
+            detail[f"cats_{int(round(s * 100))}"] = {
+                "us_per_layer": round(u, 3), "active_rows": round(float(np.mean(cnt)), 1),
+                "bytes_needed_mb": round(step_bytes(np.mean(cnt)) / 1e6, 2),
+                "achieved_gbs": round(step_bytes(np.mean(cnt)) / (u * 1e-6) / 1e9, 1),
+                "frac_of_8tbs": round(step_bytes(np.mean(cnt)) / (u * 1e-6) / 1e9 / NOMINAL_HBM_GBS, 4)}
+            del g
+        g = run_graph_steps(torch, dense_step, K, W, stream)
+        t = max_over_ranks(time_graph(g, warm_replays), world, dev)
+        u = whole_job_us_per_layer(t, K, world)
+        dense_bytes = 3.0 * 2 * H * D
+        detail["dense"] = {"us_per_layer": round(u, 3), "bytes_needed_mb": round(dense_bytes / 1e6, 2),
+                           "achieved_gbs": round(dense_bytes / (u * 1e-6) / 1e9, 1),
+                           "frac_of_8tbs": round(dense_bytes / (u * 1e-6) / 1e9 / NOMINAL_HBM_GBS, 4)}
+        detail["speedup_vs_dense"] = round(u / us, 3)
+        for key in list(detail):
+            if key.startswith("cats_"):
+                detail[key]["speedup_vs_dense"] = round(u / detail[key]["us_per_layer"], 3)
+        del g
+    del g_main
+
+    # ---- end to end through the public API: pinned host x in, host out back, every step
+    e2e = e2e_measure(torch, cs, layers, thr[args.sparsity], xs, buf, stream, K, W, world, dev)
+
+    result = {
+        "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 6), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02^2) weights, unit-RMS tokens)",
+        "config": {"workload": "llama2-7b-shaped SwiGLU FFN layer, batch-1 CATS decode",
+                   "d": D, "h": H, "batch": 1, "target_sparsity": args.sparsity,
+                   "calibration": "csffn_calibrate_threshold, 512 vectors per layer",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: steps rotate over {N_ROT} layer weight sets "
+                         f"({N_ROT * 3 * 2 * H * D / 1e9:.2f} GB)",
+                   "timing": "K steps in one CUDA graph, CUDA events on the capture stream, max over ranks"},
+        "tokens_per_s": round(world * K / (ms_max * 1e-3), 1),
+        "active_rows": round(n_act, 1),
+        "bytes_needed_mb": round(step_bytes(n_act) / 1e6, 2),
+        "achieved_gbs": round(gbs, 1),
+        "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+        f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4),
+        "roofline": {"bound": "hbm", "kernel": "gate_compact_kernel (csffn_gate_mask)",
+                     "achieved": round(gate_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "peak_source": f"{peak_kind} copy bandwidth", "frac": round(gate_gbs / peak, 4),
+                     "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": round(gate_bytes),
+                     "avg_launch_us": round(gate_avg_us, 3),
+                     "timing": "events around each launch inside the timed graph" if gate_in_graph
+                               else "events around eager launches"},
+        "e2e": e2e,
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if detail:
+        result["detail"] = detail
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.sparsity)
+    return result, rank
+
+
+def time_gate_eager(torch, cs, layers, thr, xs, buf, stream, K):
+    out = []
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            li = k % N_ROT
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            cs.gate_mask(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], thr[li], buf.idx, buf.count,
+                         buf.a_val, buf.ws)
+            b.record()
+            out.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+def e2e_measure(torch, cs, layers, thr, xs, buf, stream, K, W, world, dev):
+    """Same step through the public calls, with the token copied in from pinned host memory and the
+    output copied back to pinned host memory inside the timed region, every step."""
+    host_x = xs.cpu().pin_memory()
+    host_out = torch.empty(K, D, dtype=torch.float32).pin_memory()
+    xd = torch.empty(1, D, dtype=torch.bfloat16, device=dev)
+    od = torch.empty(1, D, dtype=torch.float32, device=dev)
+
+    def step(k, dst):
+        li = k % N_ROT
+        xd.copy_(host_x[k % N_TOKENS: k % N_TOKENS + 1], non_blocking=True)
+        cs.cats_decode(layers[li], xd, thr[li], od, buf)
+        dst.copy_(od[0], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for k in range(W):
+            step(k, host_out[k % K])
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            step(k, host_out[k])
+    torch.cuda.synchronize()
+    wall_ms = (time.perf_counter() - t0) * 1e3
+    wall_ms = max_over_ranks(wall_ms, world, dev)
+    return {"value": round(whole_job_us_per_layer(wall_ms, K, world), 3), "unit": UNIT,
+            "h2d_bytes_per_step": 2 * D, "d2h_bytes_per_step": 4 * D,
+            "how": "eager calls through the binding; host wall clock around K steps incl. pinned H2D/D2H"}
+
+
+# ---------------------------------------------------------------------------------- oracle legs
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info()]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(s: float, budget_s: float = 10.0) -> dict:
+    """The CPU oracle as it stands on this host: full 7B-shaped CATS layer calls until ~budget_s."""
+    import oracle
+    from contextual_sparsity_ffn_b200 import synth
+
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=4, n_calib=512)
+    t = oracle.calibrate_global(xc, spec, s)
+    times = []
+    t_start = time.perf_counter()
+    while len(times) < 3 or (time.perf_counter() - t_start < budget_s and len(times) < 64):
+        t0 = time.perf_counter()
+        oracle.cats_ffn(x[len(times) % 4], spec, t)
+        times.append(time.perf_counter() - t0)
+    us = 1e6 * statistics.median(times)
+    return {"value": round(us, 1), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{len(times)} full-layer oracle calls (fp64 numpy, d={D}, h={H}, batch 1), median"}
+
+
+def reference_arm(args, world, rank):
+    """The oracle timed on the host cores for the same workload, metric and unit (rank 0 only)."""
+    if rank != 0:
+        return None, rank
+    import oracle
+    from contextual_sparsity_ffn_b200 import synth
+
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=4, n_calib=512)
+    t = oracle.calibrate_global(xc, spec, args.sparsity)
+    # per-step sample: the first h_s neurons of the layer, sized so K + W steps fit ~120 s
+    t0 = time.perf_counter()
+    oracle.cats_ffn(x[0], spec, t)
+    full_s = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, budget / full_s)
+    h_s = max(64, int(H * frac))
+    sub = synth.LayerSpec(d=D, h=h_s, dtype=spec.dtype, act=spec.act, w_gate=spec.w_gate[:h_s],
+                          w_up=spec.w_up[:h_s], w_down_t=spec.w_down_t[:h_s])
+    for k in range(args.warmup):
+        oracle.cats_ffn(x[k % 4], sub, t)
+    times = []
+    for k in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.cats_ffn(x[k % 4], sub, t)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    us = 1e6 * total / args.steps * (H / h_s)
+    sample = (f"each step: oracle CATS FFN over the first {h_s} of {H} neurons (d={D}, batch 1), "
+              f"time scaled by {H / h_s:.3f} to a full layer")
+    res = {"metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "llama2-7b-shaped SwiGLU FFN layer, batch-1 CATS decode", "d": D, "h": H,
+                      "batch": 1, "target_sparsity": args.sparsity},
+           "impl": "reference",
+           "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return res, rank
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res, rank = reference_arm(args, world, rank)
+    else:
+        res, rank = csffn_arm(args, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1 and args.impl != "reference":
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

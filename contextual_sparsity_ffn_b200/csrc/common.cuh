@@ -1,0 +1,186 @@
+// Shared device helpers and the workspace layout of libcsffn.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/csffn.h"
+
+namespace csffn {
+
+typedef __nv_bfloat16 bf16;
+
+constexpr int kWarp = 32;
+
+// Device error bits recorded in the workspace error word.
+constexpr uint32_t kDevErrTimeout = 1u;
+
+// ------------------------------------------------------------------------------------------
+// Workspace layout.  The control region (counters, status words) must be zero before the first
+// call (csffn_workspace_init); every kernel that uses a counter leaves it at zero when it ends.
+// ------------------------------------------------------------------------------------------
+struct Control {           // one per compaction user, 64 bytes apart
+  uint32_t epoch;          // bumped by the last CTA of every compaction launch
+  uint32_t ticket;         // dynamic chunk tickets
+  uint32_t done;           // CTAs finished
+  uint32_t pad[13];
+};
+
+constexpr int kCtlGate = 0;     // csffn_gate_mask
+constexpr int kCtlPred = 1;     // csffn_predict_lowrank
+constexpr int kNumCtl = 4;
+constexpr int kMaxSlices = 128;  // column slices of the down projection (d / slice width)
+constexpr int kMaxRowRanges = 64;
+constexpr int kSliceUsers = 2;  // sparse forward, dense forward
+
+struct WsLayout {
+  size_t ctl;        // Control[kNumCtl]
+  size_t err;        // uint32 error word (+ pad)
+  size_t slice_ctr;  // uint32 [kSliceUsers][kMaxSlices]
+  size_t status;     // uint64 [kNumCtl][max_chunks]   look-back status words
+  size_t control_end;
+  size_t vbuf;       // fp32 [max_batch][h]            v = a * u (sparse) or act(z)*u (dense)
+  size_t partial;    // fp32 [kMaxRowRanges][max_batch][d]
+  size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
+  size_t total;
+  int max_chunks;
+};
+
+constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
+  WsLayout L;
+  size_t o = 0;
+  L.ctl = o;        o += sizeof(Control) * kNumCtl;
+  L.err = o;        o += 64;
+  L.slice_ctr = o;  o += sizeof(uint32_t) * kSliceUsers * kMaxSlices;
+  o = align_up(o, 256);
+  L.max_chunks = (h + kChunkRows - 1) / kChunkRows;
+  L.status = o;     o += sizeof(uint64_t) * (size_t)kNumCtl * L.max_chunks;
+  o = align_up(o, 256);
+  L.control_end = o;
+  L.vbuf = o;       o += sizeof(float) * (size_t)max_batch * h;
+  o = align_up(o, 256);
+  L.partial = o;    o += sizeof(float) * (size_t)kMaxRowRanges * max_batch * d;
+  o = align_up(o, 256);
+  L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);
+  o = align_up(o, 256);
+  L.total = o;
+  return L;
+}
+
+// The layout is recomputed from (d, h, B, rank) on every call.  The control region's offsets
+// depend on h only, so counters persist correctly across calls with different batch sizes; the
+// scratch regions after it are per call.  Each entry point checks ws_bytes against its needs.
+
+// ------------------------------------------------------------------------------------------
+// Loads and conversions
+// ------------------------------------------------------------------------------------------
+
+// Streaming 16-byte load of read-once weights: read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <typename T> struct Vec;
+template <> struct Vec<bf16> { static constexpr int N = 8; };
+template <> struct Vec<float> { static constexpr int N = 4; };
+
+// 16 bytes of weights -> N floats.
+__device__ __forceinline__ void unpack(const uint4& w, float (&f)[8]) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+__device__ __forceinline__ void unpack(const uint4& w, float (&f)[4]) {
+  f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+  f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+}
+
+// N consecutive x values from shared memory (16-byte aligned), as floats.
+template <int N>
+__device__ __forceinline__ void load_x(const bf16* p, float (&f)[N]) {
+  static_assert(N == 8, "bf16 x pairs with bf16 weights");
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  unpack(v, f);
+}
+template <int N>
+__device__ __forceinline__ void load_x(const float* p, float (&f)[N]) {
+  if constexpr (N == 8) {
+    float4 a = reinterpret_cast<const float4*>(p)[0];
+    float4 b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  } else {
+    float4 a = reinterpret_cast<const float4*>(p)[0];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// SwiGLU / ReGLU gate activation.  SiLU(z) = z / (1 + e^-z), with CUDA's expf.
+__device__ __forceinline__ float gate_act(float z, int act) {
+  return act == CSFFN_ACT_SILU ? z / (1.0f + expf(-z)) : fmaxf(z, 0.0f);
+}
+
+// ------------------------------------------------------------------------------------------
+// Acquire/release accesses for cross-CTA status words
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t ld_acquire(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Look-back status word: [epoch:32 | flag:2 | value:30].
+constexpr uint64_t kFlagAggregate = 1, kFlagInclusive = 2;
+__device__ __forceinline__ uint64_t status_word(uint32_t epoch, uint64_t flag, uint32_t value) {
+  return ((uint64_t)epoch << 32) | (flag << 30) | (uint64_t)value;
+}
+
+// Polls before a bounded wait gives up: 2^22 polls with ~128 ns sleeps (about half a second),
+// far beyond any wait on a CTA that is running.
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+// Bounded wait on a 64-bit status word: polls *p (acquire) until ready(value) holds or `limit`
+// polls have failed.  On success returns true with the word in *out; on give-up records
+// kDevErrTimeout in *err and returns false.  Every device-side wait in the library uses this.
+template <typename Ready>
+__device__ __forceinline__ bool bounded_wait(const uint64_t* p, uint32_t limit, uint32_t* err,
+                                             Ready ready, uint64_t* out) {
+  for (uint32_t spins = 0;; ++spins) {
+    const uint64_t v = ld_acquire(p);
+    if (ready(v)) {
+      *out = v;
+      return true;
+    }
+    if (spins >= limit) {
+      atomicOr(err, kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(128);
+  }
+}
+
+}  // namespace csffn

@@ -1,0 +1,102 @@
+// Host-side launchers of libcsffn's kernels (internal; the public surface is include/csffn.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csffn {
+
+struct Control;
+
+// Token-capacity tier used to instantiate the GEMV kernels: 1, 2, 4, 8 or 16.
+inline int batch_tier(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
+
+enum GateMode { kModeCats = 0, kModePred = 1 };
+
+// Fused row GEMV + activation/compare + union over tokens + ascending compaction.
+struct GateArgs {
+  const void* W;              // [h, K] rows (W_gate, or V_r for the predictor)
+  const void* x;              // [B, K] tokens: weight dtype (CATS) or fp32 (predictor y)
+  int K, h, B;
+  const float* bias;          // [h] or NULL
+  float t;                    // CATS threshold on |act(z)|
+  const float* tau;           // [h] per-neuron thresholds on z (predictor mode)
+  int act;                    // csffn_act
+  const int32_t* cand_idx;    // NULL = rows 0..h-1
+  const int32_t* cand_count;
+  int32_t* idx;
+  int32_t* count;
+  float* a_val;               // [B, h] (CATS mode)
+  Control* ctl;
+  uint64_t* status;
+  uint32_t* err;
+};
+cudaError_t launch_gate_compact(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
+
+// v[b*h + j] = a_val[b*h + j] * (x_b . W_up[idx[j]]) for j < *count.
+struct UpArgs {
+  const void* W_up;
+  const void* x;
+  int d, h, B;
+  const int32_t* idx;
+  const int32_t* count;
+  const float* a_val;
+  float* v;
+};
+cudaError_t launch_up_gather(const UpArgs& a, int wdtype, cudaStream_t s);
+
+// v[b*h + i] = act(x_b . W_gate[i] + beta_i) * (x_b . W_up[i]) for all i < h.
+struct DenseGateUpArgs {
+  const void* W_gate;
+  const void* W_up;
+  const void* x;
+  int d, h, B;
+  const float* bias;
+  int act;
+  float* v;
+};
+cudaError_t launch_dense_gate_up(const DenseGateUpArgs& a, int wdtype, cudaStream_t s);
+
+// out[b, :] (=|+=) sum_{j < n} v[b*h + j] * W_down^T[idx ? idx[j] : j, :]
+struct DownArgs {
+  const void* W_down_t;
+  int d, h, B;
+  const int32_t* idx;     // NULL = identity
+  const int32_t* count;   // NULL = n_host
+  int n_host;
+  const float* v;
+  float* partial;         // [row_ranges][B][d]
+  uint32_t* slice_ctr;    // [slices]
+  void* out;
+  int out_mode;
+};
+cudaError_t launch_down_gather(const DownArgs& a, int wdtype, cudaStream_t s);
+
+// y[b*rank + k] = x_b . U_r^T[k]  (plain GEMV, fp32 out)
+struct RowGemvArgs {
+  const void* W;      // [rows, K]
+  const void* x;      // [B, K] weight dtype
+  int rows, K, B;
+  float* y;           // [B, rows]   (y[b*y_stride + row])
+  int y_stride;
+  const float* bias;  // [rows] or NULL, added
+  int act;            // -1 = none, else csffn_act
+  int abs_out;        // write |value|
+  int transpose_out;  // write y[row*y_stride + b] instead
+};
+cudaError_t launch_row_gemv(const RowGemvArgs& a, int wdtype, bool x_f32, cudaStream_t s);
+
+// Radix selection and per-neuron selection (calibration).
+size_t kth_state_bytes();
+cudaError_t launch_kth_smallest(const float* values, int64_t n, int64_t k, float* out, void* state,
+                                cudaStream_t s);
+cudaError_t launch_rows_kth(const float* values, int rows, int n, int k, float* out, cudaStream_t s);
+cudaError_t launch_fill(float* p, float v, int n, cudaStream_t s);
+
+cudaError_t launch_rmsnorm_bf16(const float* h, int B, int d, float eps, void* xn, cudaStream_t s);
+
+cudaError_t launch_timeout_selftest(uint64_t* flag, uint32_t* err, int spin_limit, cudaStream_t s);
+
+int sm_count();
+
+}  // namespace csffn

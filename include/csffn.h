@@ -1,0 +1,205 @@
+/*
+ * csffn -- contextually sparse gated FFN at decode time, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libcsffn.so.  Plain pointers and sizes only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument named x, w_*, idx, count, a_val, out, t_out, tau,
+ *    u_rt, v_r, values, ws is a DEVICE pointer owned by the caller.  The library
+ *    keeps no pointer after the call returns and allocates no device memory on
+ *    any path: scratch space comes from a caller workspace (`ws`) whose size is
+ *    queried up front.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream; nothing synchronises except
+ *    csffn_check_status.  Index counts (`count`, `cand_count`) stay in device
+ *    memory, so a whole decode step can be captured in a CUDA graph.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call launches nothing and returns the error.  Nothing throws.
+ *  - Device-side errors (a bounded wait that ran out) are recorded in an error
+ *    word inside the workspace and reported by csffn_check_status.
+ *  - One workspace must not be used by two streams at once: calls that share a
+ *    workspace must be ordered on one stream.
+ *  - Weights are neuron-major: W_gate and W_up are [h, d] (row i = neuron i's
+ *    input weights, the nn.Linear [out, in] layout) and W_down^T is [h, d]
+ *    (row i = neuron i's output weights, i.e. the down projection [d, h]
+ *    transposed).  Skipping a neuron therefore skips whole contiguous rows.
+ *  - Token vectors x are [B, d] row-major in the weight dtype.
+ *  - Alignment: d % 8 == 0 for bf16, d % 4 == 0 for fp32; every weight, x and
+ *    out pointer 16-byte aligned; otherwise CSFFN_ERR_ALIGNMENT.
+ *  - Index lists (idx, cand_idx) are int32, unique and ascending.
+ *  - Batch limits: 1 <= B <= CSFFN_MAX_BATCH (B == 0 is an empty call, see each
+ *    function).  Shape limits: 1 <= h <= CSFFN_MAX_H, 8 <= d <= CSFFN_MAX_D.
+ *
+ * Sources (page titles; figure/section on each page):
+ *  [CATS]   "CATS: Contextually-Aware Thresholding for Sparsity in Large Language
+ *           Models", abstract -- thresholded SiLU gate activation; a GPU kernel
+ *           fusing the gate GEMV with the compare and a flag-gated GEMV.
+ *  [SVDP]   "SVD Contextual Sparsity Predictors for Fast LLM Inference", abstract,
+ *           Fig. 1 (offline SVD predictors + calibrated per-neuron thresholds run
+ *           ahead of each FFN), Fig. 3 (ReGLU: gate then up run sequentially on the
+ *           predicted-active neurons), Table 3 ("+ Bias calibration").
+ *  [SIRIUS] "Sirius: Contextual Sparsity with Correction for Efficient LLMs",
+ *           abstract and its summary page, "Approach" -- sparse and full model
+ *           share weights; the full model verifies a chunk of tokens in parallel.
+ */
+#ifndef CSFFN_H
+#define CSFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSFFN_VERSION 1
+#define CSFFN_MAX_BATCH 16
+#define CSFFN_MAX_D 16384
+#define CSFFN_MAX_H (1 << 24)
+#define CSFFN_MAX_RANK 4096
+#define CSFFN_MAX_CALIB 8192
+
+typedef enum {
+  CSFFN_OK = 0,
+  CSFFN_ERR_INVALID_ARG = 1,       /* NULL pointer, bad enum, B/n/k/rank out of range */
+  CSFFN_ERR_UNSUPPORTED_SHAPE = 2, /* d/h/B combination this build does not run */
+  CSFFN_ERR_ALIGNMENT = 3,         /* d not a multiple of the vector width, or pointer not 16-B aligned */
+  CSFFN_ERR_WORKSPACE = 4,         /* ws NULL or ws_bytes below the queried size */
+  CSFFN_ERR_CUDA = 5,              /* a CUDA runtime call or kernel launch failed */
+  CSFFN_ERR_TIMEOUT = 6            /* a bounded device-side wait ran out (see csffn_check_status) */
+} csffn_status;
+
+typedef enum { CSFFN_BF16 = 0, CSFFN_F32 = 1 } csffn_dtype;
+
+/* Output modes of the forward calls: write bf16, write fp32, or add into an fp32
+ * buffer (out += FFN(x), the residual update of a transformer block). */
+typedef enum { CSFFN_OUT_BF16 = 0, CSFFN_OUT_F32 = 1, CSFFN_OUT_F32_ACCUMULATE = 2 } csffn_out_mode;
+
+/* SILU: SwiGLU gate a = SiLU(z); RELU: ReGLU gate a = max(z, 0).  z = x.W_gate[i] + beta_i. */
+typedef enum { CSFFN_ACT_SILU = 0, CSFFN_ACT_RELU = 1 } csffn_act;
+
+typedef enum {
+  CSFFN_CAL_GLOBAL_ABS_ACT = 0,  /* one scalar t: quantile of |a| over calibration set x neurons [CATS] */
+  CSFFN_CAL_PER_NEURON_PRED = 1  /* tau[h]: per-neuron quantile of the SVD predictor output [SVDP] Fig. 1 */
+} csffn_cal_mode;
+
+/* One gated FFN layer.  wdtype applies to w_gate, w_up, w_down_t and to x. */
+typedef struct {
+  int32_t d;              /* model (hidden) width */
+  int32_t h;              /* FFN intermediate width = number of neurons */
+  int32_t wdtype;         /* csffn_dtype */
+  int32_t act;            /* csffn_act */
+  const void* w_gate;     /* [h, d] */
+  const void* w_up;       /* [h, d] */
+  const void* w_down_t;   /* [h, d] */
+  const float* gate_bias; /* [h] fp32 added to z, or NULL */
+} csffn_layer;
+
+/* Library version (CSFFN_VERSION). */
+int csffn_version(void);
+
+/* Static string for a status code. */
+const char* csffn_status_string(int status);
+
+/* Bytes of workspace the decode-path calls need for this layer at batch
+ * <= max_batch and predictor rank <= max_rank (0 if no predictor is used).
+ * Returns 0 if the arguments are invalid. */
+size_t csffn_workspace_size(const csffn_layer* layer, int max_batch, int max_rank);
+
+/* Zero the workspace's control words; required once before first use and after
+ * a CSFFN_ERR_TIMEOUT.  Asynchronous on `stream`. */
+csffn_status csffn_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the device-side error word of `ws`.
+ * Returns CSFFN_OK, CSFFN_ERR_TIMEOUT (a bounded wait ran out: re-initialise the
+ * workspace with csffn_workspace_init before reuse) or CSFFN_ERR_CUDA. */
+csffn_status csffn_check_status(void* ws, void* stream);
+
+/* Gate GEMV + activation + threshold + active-index compaction (one kernel).
+ * [CATS] abstract (fused gate GEMV + compare + flag); [SVDP] Fig. 3 (gate on the
+ * predicted set).
+ *   z[b,i] = x_b . W_gate[i,:] + beta_i,  a = act(z),  token b keeps neuron i iff |a[b,i]| > t.
+ *   Rows considered: all h neurons if cand_idx == NULL, else cand_idx[0 .. *cand_count).
+ *   Outputs: idx[0 .. *count) = ascending indices of neurons kept by ANY token (the
+ *   union over the batch); a_val[b*h + j] = a[b, idx[j]] if token b keeps idx[j],
+ *   else 0 (per-token values, union rows).  idx: int32 [h]; count: int32 [1];
+ *   a_val: fp32 [B, h] (row stride h; entries j >= *count are untouched).
+ *   With act = RELU and t = 0 the kept set is {z > 0}.  t may be negative (keeps all).
+ *   B == 0: writes *count = 0 and nothing else. */
+csffn_status csffn_gate_mask(const csffn_layer* layer, const void* x, int B, float t,
+                             const int32_t* cand_idx, const int32_t* cand_count,
+                             int32_t* idx, int32_t* count, float* a_val,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Gathered up- and down-projection over the active rows.  [CATS] abstract
+ * (flag-gated GEMV); [SVDP] Fig. 3 (up and down only on the active set).
+ *   out[b,:] = sum_{j < *count} a_val[b*h + j] * (x_b . W_up[idx[j],:]) * W_down^T[idx[j],:]
+ *   Reads only rows idx[0 .. *count) of W_up and W_down^T.  *count is read on the
+ *   device.  out: [B, d] in the dtype of out_mode (ACCUMULATE adds into fp32 out).
+ *   *count == 0 gives out = 0 (or leaves an accumulated out unchanged).  B == 0: no-op. */
+csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, int B,
+                                      const int32_t* idx, const int32_t* count, const float* a_val,
+                                      void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* Dense gated FFN over all h neurons (the full model that verifies a chunk of
+ * sparse-drafted tokens, [SIRIUS] "Approach"; also the speed-up baseline).
+ *   out = (act(x W_gate^T + beta) * (x W_up^T)) W_down.  B == 0: no-op.
+ *   bf16 layers with B >= 8 run on the tensor cores (the 16-token verify chunk);
+ *   their intermediate activations are rounded to bf16 before the down GEMM. */
+csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,
+                                     void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* SVD low-rank predictor + per-neuron compare + compaction.  [SVDP] Fig. 1.
+ *   y = x U_r (u_rt is U_r^T, [rank, d], row k = sigma_k * k-th left singular vector),
+ *   p[b,i] = y_b . V_r[i,:] + beta_i (v_r: [h, rank]; beta = layer->gate_bias or 0),
+ *   neuron i is a candidate iff p[b,i] > tau[i] for ANY token b.
+ *   cand_idx[0 .. *cand_count) = ascending candidates (int32 [h]; count int32 [1]).
+ *   u_rt, v_r in layer->wdtype; rank % (8 for bf16, 4 for fp32) == 0.
+ *   B == 0: writes *cand_count = 0. */
+csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int B, int rank,
+                                   const void* u_rt, const void* v_r, const float* tau,
+                                   int32_t* cand_idx, int32_t* cand_count,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes for csffn_calibrate_threshold with n calibration vectors. */
+size_t csffn_calibrate_workspace_size(const csffn_layer* layer, int n, int mode, int rank);
+
+/* Offline threshold calibration.  [CATS] abstract (contextually-aware threshold);
+ * [SVDP] Fig. 1, Table 3 ("bias calibration").
+ *   GLOBAL_ABS_ACT: M = n*h values |act(z)| over x_cal [n, d]; k = ceil(s*M) with s
+ *     taken as this float and the product evaluated exactly; *t_out = v_(k)
+ *     (k-th smallest, 1-indexed), or 0 when k == 0.
+ *   PER_NEURON_PRED: p as in csffn_predict_lowrank for each calibration vector;
+ *     k = ceil(s*n); t_out[i] = k-th smallest of {p_i(x_n)} (t_out is [h]), or
+ *     -inf when k == 0.
+ *   1 <= n <= CSFFN_MAX_CALIB, 0 <= s <= 1. */
+csffn_status csffn_calibrate_threshold(const csffn_layer* layer, const void* x_cal, int n,
+                                       float target_sparsity, int mode,
+                                       const void* u_rt, const void* v_r, int rank,
+                                       float* t_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Exact k-th smallest (1 <= k <= n) of n finite fp32 values by radix selection on
+ * their order-preserving bit keys; *out receives the selected value bit-exactly.
+ * Building block of GLOBAL_ABS_ACT calibration.  ws: csffn_kth_workspace_size(). */
+size_t csffn_kth_workspace_size(void);
+csffn_status csffn_kth_smallest(const float* values, int64_t n, int64_t k, float* out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* RMSNorm with unit gain, rounded to bf16: xn[b,:] = bf16(h[b,:] / sqrt(mean(h[b,:]^2) + eps)).
+ * h: fp32 [B, d]; xn: bf16 [B, d].  The input step of each block of an FFN stack
+ * (h <- h + FFN(RMSNorm(h)) with out_mode ACCUMULATE). */
+csffn_status csffn_rmsnorm_bf16(const float* h, int B, int d, float eps, void* xn, void* stream);
+
+/* Failure-detection self-test: launches one tiny kernel that waits, with the same
+ * bounded wait the look-back compaction uses, on a workspace flag that nothing
+ * sets.  After `spin_limit` polls it records CSFFN_ERR_TIMEOUT in the workspace
+ * error word and returns; csffn_check_status then reports it.  The context stays
+ * usable.  Run csffn_workspace_init afterwards. */
+csffn_status csffn_selftest_timeout(void* ws, size_t ws_bytes, int spin_limit, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSFFN_H */

@@ -1,0 +1,168 @@
+"""CUDA path vs the CPU oracle: threshold calibration, the SVD low-rank predictor, the gathered
+gate on the predicted set and the sequential ReGLU FFN."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from contextual_sparsity_ffn_b200 import synth
+from contextual_sparsity_ffn_b200 import binding as cs
+from contextual_sparsity_ffn_b200 import _abi
+
+from gpu_helpers import assert_index_list, dev, dev_layer, run_gate, run_sparse
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------------------ order statistics
+
+@pytest.mark.parametrize("n,ks", [(1, [1]), (1000, [1, 500, 1000]), (5_636_096, [2_818_048, 3_945_268, 5_072_487])])
+def test_kth_smallest_bit_exact(n, ks):
+    rng = np.random.default_rng(n)
+    v = (np.abs(rng.standard_normal(n)) * 0.3).astype(np.float32)
+    v[: min(n, 50)] = v[0]  # ties
+    vs = np.sort(v)
+    vals = torch.from_numpy(v).cuda()
+    out = torch.zeros(1, device="cuda")
+    for k in ks:
+        cs.kth_smallest(vals, k, out)
+        got = out.cpu().numpy()[0]
+        assert got.view(np.uint32) == vs[k - 1].view(np.uint32)
+
+
+def test_kth_smallest_signed_values():
+    v = np.array([3.5, -1.0, 0.0, -0.0, 2.0, -7.25, 1e-30, -1e-30], np.float32)
+    vals = torch.from_numpy(v).cuda()
+    out = torch.zeros(1, device="cuda")
+    for k in range(1, len(v) + 1):
+        cs.kth_smallest(vals, k, out)
+        assert out.item() == np.sort(v)[k - 1]
+
+
+def test_kth_on_oracle_activations_bit_exact():
+    spec, _, xc = synth.tiny_swiglu()
+    vals = np.abs(oracle.gate_activation(xc, spec)).ravel().astype(np.float32)
+    k = oracle.order_statistic_rank(0.5, vals.size)
+    out = torch.zeros(1, device="cuda")
+    cs.kth_smallest(torch.from_numpy(vals).cuda(), k, out)
+    assert out.cpu().numpy()[0].view(np.uint32) == np.sort(vals)[k - 1].view(np.uint32)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.7, 0.9, 1.0])
+def test_calibrate_global_tiny(s):
+    spec, _, xc = synth.tiny_swiglu()
+    layer = dev_layer(spec)
+    t_out = torch.zeros(1, device="cuda")
+    cs.calibrate_threshold(layer, dev(xc), s, _abi.CAL_GLOBAL_ABS_ACT, t_out)
+    t_ref = oracle.calibrate_global(xc, spec, s)
+    assert t_out.item() == pytest.approx(t_ref, rel=1e-5, abs=1e-7)
+
+
+@pytest.mark.parametrize("s", [0.5, 0.7, 0.9])
+def test_calibrate_global_7b(s):
+    spec, _, xc = synth.llama2_7b_swiglu(0, n_eval=1, n_calib=512)
+    layer = dev_layer(spec)
+    t_out = torch.zeros(1, device="cuda")
+    cs.calibrate_threshold(layer, dev(xc), s, _abi.CAL_GLOBAL_ABS_ACT, t_out)
+    a = np.abs(oracle.gate_activation(xc, spec))
+    t_ref = oracle.calibrate_global(xc, spec, s)
+    assert t_out.item() == pytest.approx(t_ref, rel=1e-5)
+    # the GPU's t hits the requested sparsity on the calibration set
+    frac = float((a <= t_out.item()).mean())
+    assert abs(frac - s) < 1e-4
+
+
+# ------------------------------------------------------------------------------ SVD predictor
+
+@functools.lru_cache(maxsize=None)
+def reglu_case(d, h, r, n_calib, q=0.9):
+    """Workload-2 style layer with oracle SVD factors rounded to bf16 (inputs to both sides)."""
+    spec, x, xc = synth.reglu_sparse(0, d=d, h=h, n_eval=4, n_calib=n_calib)
+    urt, vr = oracle.svd_factors(spec.w_gate, r)
+    urt_b = synth.bf16_bits(urt.astype(np.float32))
+    vr_b = synth.bf16_bits(vr.astype(np.float32))
+    tau = oracle.calibrate_per_neuron(xc, urt_b, vr_b, spec.bias, q)
+    return spec, x, xc, urt_b, vr_b, tau
+
+
+def _pred_band(p, tau, rms):
+    return (np.abs(p - tau[None, :]) < 1e-3 * np.maximum(np.abs(tau), rms)[None, :]).any(axis=0)
+
+
+@pytest.mark.parametrize("d,h,r", [(1024, 2048, 128), (4096, 11008, 256), (4096, 11008, 1024)])
+def test_per_neuron_calibration(d, h, r):
+    spec, x, xc, urt, vr, tau_ref = reglu_case(d, h, r, 512)
+    layer = dev_layer(spec)
+    tau = torch.zeros(h, device="cuda")
+    cs.calibrate_threshold(layer, dev(xc), 0.9, _abi.CAL_PER_NEURON_PRED, tau, u_rt=dev(urt), v_r=dev(vr))
+    p = oracle.predict(xc, urt, vr, spec.bias)
+    rms = np.sqrt(np.mean(p * p, axis=0))
+    np.testing.assert_allclose(tau.cpu().numpy(), tau_ref, rtol=1e-4, atol=1e-5 * rms.max())
+
+
+@pytest.mark.parametrize("d,h,r", [(1024, 2048, 128), (4096, 11008, 256), (4096, 11008, 1024)])
+@pytest.mark.parametrize("B", [1, 4])
+def test_predict_gate_reglu_sequential(d, h, r, B):
+    spec, x, xc, urt, vr, tau_ref = reglu_case(d, h, r, 512)
+    x = x[:B]
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, B, r)
+    tau = torch.from_numpy(tau_ref.astype(np.float32)).cuda()
+    tau64 = tau.cpu().numpy().astype(np.float64)
+    cand_idx = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cand_count = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xd = dev(x)
+    cs.predict_lowrank(layer, xd, dev(urt), dev(vr), tau, cand_idx, cand_count, ws)
+    assert cs.check_status(ws) == 0
+    nP = int(cand_count.item())
+    P = cand_idx[:nP].cpu().numpy()
+    assert_index_list(P, h)
+    # predicted set vs oracle, outside the band
+    p = oracle.predict(x, urt, vr, spec.bias)
+    p_cal = oracle.predict(xc, urt, vr, spec.bias)
+    rms = np.sqrt(np.mean(p_cal * p_cal, axis=0))
+    pm_ref = oracle.union_mask(oracle.predicted_mask(p, tau64))
+    band = _pred_band(p, tau64, rms)
+    got = np.zeros(h, bool)
+    got[P] = True
+    assert np.array_equal(got[~band], pm_ref[~band])
+    assert 0.02 < nP / h < (0.5 if B == 1 else 0.9)
+    # gathered gate on P (ReLU, t = 0), then up/down on A
+    idx, a_val, bufs = run_gate(layer, x, 0.0, ws=ws, cand=(cand_idx, cand_count))
+    assert_index_list(idx, h)
+    assert set(idx.tolist()) <= set(P.tolist())
+    z = oracle.gate_preactivation(x, spec)
+    zrms = np.sqrt(np.mean(z * z))
+    amask_gpu = np.zeros((B, h), bool)
+    amask_gpu[:, idx] = a_val != 0.0
+    pred_tok = np.zeros((B, h), bool)
+    pred_tok[:, P] = True  # union of predicted rows: every token's gate runs on it
+    a_ref = pred_tok & (z > 0)
+    clear = np.abs(z) > 1e-3 * zrms
+    assert np.array_equal(amask_gpu[clear], a_ref[clear])
+    out = run_sparse(layer, bufs)
+    ref, _ = oracle.reglu_sequential(x, spec, amask_gpu)
+    assert oracle.rel_l2(out, ref) <= 1e-4
+
+
+def test_predictor_full_rank_is_the_gate():
+    """At full rank the predicted set with tau = 0 is {z > 0} (up to bf16 factor rounding)."""
+    d, h = 256, 512
+    spec = synth.make_layer(57, 0, d, h, "bf16", "relu", bias_mean_std=(-0.3, 0.1))
+    x = synth.make_tokens(57, 0, synth.ROLE_EVAL, 1, d, "bf16", rms_normalise=True)
+    urt, vr = oracle.svd_factors(spec.w_gate, d)
+    urt_b, vr_b = synth.bf16_bits(urt.astype(np.float32)), synth.bf16_bits(vr.astype(np.float32))
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 1, d)
+    tau = torch.zeros(h, device="cuda")
+    ci = torch.zeros(h, dtype=torch.int32, device="cuda")
+    cc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cs.predict_lowrank(layer, dev(x), dev(urt_b), dev(vr_b), tau, ci, cc, ws)
+    P = ci[: int(cc.item())].cpu().numpy()
+    z = oracle.gate_preactivation(x, spec)[0]
+    got = np.zeros(h, bool)
+    got[P] = True
+    clear = np.abs(z) > 0.05 * np.sqrt(np.mean(z * z))
+    assert np.array_equal(got[clear], (z > 0)[clear])

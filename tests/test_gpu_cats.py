@@ -1,0 +1,217 @@
+"""CUDA path vs the CPU oracle: CATS gate mask, gathered sparse FFN, dense FFN, union of masks.
+
+Parity rules: the active-index set is bit-exact outside the band ||a| - t| < 1e-3 t; the output is
+then compared with the oracle run on the GPU's own per-token mask.  Max relative L2 error per
+output vector: <= 1e-5 for fp32 workloads, <= 1e-2 for bf16 workloads (plus a tighter 1e-4 check
+on fp32 outputs of bf16 layers, which any single dropped or wrong neuron would exceed).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from contextual_sparsity_ffn_b200 import synth
+from contextual_sparsity_ffn_b200 import binding as cs
+
+from gpu_helpers import (assert_index_list, band_rows, dev, dev_layer, run_dense, run_gate, run_sparse,
+                         token_masks)
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-2
+TOL_BF16_F32OUT = 1e-4
+
+
+def check_cats(spec, x, t, tol, layer=None, out_dtype=torch.float32):
+    """Run gate + sparse forward on the GPU and check against the oracle; return (err, density)."""
+    layer = layer or dev_layer(spec)
+    idx, a_val, bufs = run_gate(layer, x, t)
+    assert_index_list(idx, spec.h)
+    a_ref = oracle.gate_activation(x, spec)
+    m_ref = oracle.cats_mask(a_ref, t)
+    union_ref = oracle.union_mask(m_ref)
+    band = band_rows(a_ref, t)
+    got = np.zeros(spec.h, dtype=bool)
+    got[idx] = True
+    assert np.array_equal(got[~band], union_ref[~band]), "active set differs outside the band"
+    # per-token values: a where the token keeps the neuron, else 0
+    m_gpu = token_masks(idx, a_val, spec.h)
+    tb = np.abs(np.abs(a_ref) - t) < 1e-3 * abs(t)
+    assert np.array_equal(m_gpu[~tb], m_ref[~tb])
+    a_sel = np.where(m_gpu, a_ref, 0.0)[:, idx]
+    np.testing.assert_allclose(a_val, a_sel, rtol=1e-4, atol=1e-6 * np.abs(a_ref).max())
+    out = run_sparse(layer, bufs, out_dtype=out_dtype)
+    ref = oracle.sparse_ffn(x, spec, m_gpu)
+    err = oracle.rel_l2(out, ref)
+    assert err <= tol, f"rel L2 {err:.3e} > {tol}"
+    return err, len(idx) / spec.h, out
+
+
+# ------------------------------------------------------------------------------ tiny fp32 workload
+
+def test_tiny_fp32_each_token():
+    spec, x, xc = synth.tiny_swiglu()
+    t = oracle.calibrate_global(xc, spec, 0.5)
+    layer = dev_layer(spec)
+    for b in range(x.shape[0]):
+        err, dens, _ = check_cats(spec, x[b:b + 1], t, TOL_F32, layer=layer)
+        assert 0.3 < dens < 0.7
+
+
+def test_tiny_fp32_union_batch16():
+    spec, x, xc = synth.tiny_swiglu()
+    t = oracle.calibrate_global(xc, spec, 0.5)
+    err, dens, out = check_cats(spec, x, t, TOL_F32)
+    assert dens > 0.99  # union of 16 independent tokens at 50% is ~1 - 2^-16
+    # batched output == each token alone
+    layer = dev_layer(spec)
+    for b in [0, 7, 15]:
+        _, _, ob = check_cats(spec, x[b:b + 1], t, TOL_F32, layer=layer)
+        assert oracle.rel_l2(out[b], ob[0]) <= TOL_F32
+
+
+def test_tiny_fp32_dense():
+    spec, x, _ = synth.tiny_swiglu()
+    out = run_dense(dev_layer(spec), x)
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_F32
+
+
+# ------------------------------------------------------------------------------ ragged shapes
+
+@pytest.mark.parametrize("d,h,B", [(520, 1000, 1), (520, 1000, 3), (8, 5, 1), (64, 16, 2), (1032, 33, 5),
+                                   (4104, 777, 1)])
+def test_ragged_bf16(d, h, B):
+    spec = synth.make_layer(50, d, d, h, "bf16")
+    x = synth.make_tokens(50, d, synth.ROLE_EVAL, B, d, "bf16", rms_normalise=True)
+    a = np.abs(oracle.gate_activation(x, spec))
+    t = float(np.quantile(a, 0.5))
+    check_cats(spec, x, t, TOL_BF16_F32OUT)
+    out = run_dense(dev_layer(spec), x)
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16_F32OUT
+
+
+@pytest.mark.parametrize("d,h", [(256, 688), (12, 40)])
+def test_ragged_fp32(d, h):
+    spec = synth.make_layer(51, d, d, h, "f32")
+    x = synth.make_tokens(51, d, synth.ROLE_EVAL, 2, d, "f32", rms_normalise=False)
+    t = float(np.quantile(np.abs(oracle.gate_activation(x, spec)), 0.7))
+    check_cats(spec, x, t, TOL_F32)
+
+
+# ------------------------------------------------------------------------------ degenerate cases
+
+def test_empty_active_set_gives_zero():
+    spec = synth.make_layer(52, 0, 256, 300, "bf16")
+    x = synth.make_tokens(52, 0, synth.ROLE_EVAL, 2, 256, "bf16", rms_normalise=True)
+    layer = dev_layer(spec)
+    idx, a_val, bufs = run_gate(layer, x, 1e9)
+    assert len(idx) == 0
+    out = run_sparse(layer, bufs)
+    assert np.all(out == 0.0)
+    # accumulate mode leaves the residual unchanged
+    res = torch.arange(2 * 256, dtype=torch.float32, device="cuda").reshape(2, 256)
+    keep = res.clone()
+    cs.sparse_ffn_forward(layer, bufs["x"], bufs["idx"], bufs["count"], bufs["a_val"], res, bufs["ws"],
+                          out_mode=cs._abi.OUT_F32_ACCUMULATE)
+    assert torch.equal(res, keep)
+
+
+def test_all_active_equals_dense():
+    spec, x, _ = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=1)
+    layer = dev_layer(spec)
+    idx, a_val, bufs = run_gate(layer, x, -1.0)
+    assert len(idx) == spec.h
+    out = run_sparse(layer, bufs)
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16_F32OUT
+    assert oracle.rel_l2(out, run_dense(layer, x)) <= TOL_BF16_F32OUT
+
+
+def test_reglu_t0_equals_dense():
+    spec = synth.make_layer(53, 0, 1024, 2000, "bf16", "relu", bias_mean_std=(-0.5, 0.2))
+    x = synth.make_tokens(53, 0, synth.ROLE_EVAL, 1, 1024, "bf16", rms_normalise=True)
+    layer = dev_layer(spec)
+    idx, a_val, bufs = run_gate(layer, x, 0.0)
+    z = oracle.gate_preactivation(x, spec)[0]
+    clear = np.abs(z) > 1e-4
+    got = np.zeros(spec.h, bool)
+    got[idx] = True
+    assert np.array_equal(got[clear], (z > 0)[clear])
+    out = run_sparse(layer, bufs)
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16_F32OUT
+
+
+def test_batch_zero_writes_zero_count():
+    spec = synth.make_layer(54, 0, 64, 40, "bf16")
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 1)
+    count = torch.full((1,), 5, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(40, dtype=torch.int32, device="cuda")
+    a_val = torch.zeros(1, 40, device="cuda")
+    x = torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda")
+    cs._abi.check(cs.load().csffn_gate_mask(layer.ref(), None, 0, 0.1, None, None, cs._ptr(idx), cs._ptr(count),
+                                            cs._ptr(a_val), cs._ptr(ws), ws.numel(), cs._stream()), "b0")
+    assert int(count.item()) == 0
+
+
+def test_repeated_calls_reuse_workspace():
+    """Epoch-tagged look-back: many launches on one workspace give identical results."""
+    spec = synth.make_layer(55, 0, 512, 3000, "bf16")
+    x = synth.make_tokens(55, 0, synth.ROLE_EVAL, 1, 512, "bf16", rms_normalise=True)
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 4)
+    first = None
+    for it in range(20):
+        t = 0.05 if it % 2 == 0 else 0.2
+        idx, a_val, bufs = run_gate(layer, x, t, ws=ws)
+        out = run_sparse(layer, bufs)
+        if it < 2:
+            first = first or {}
+            first[t] = (idx.copy(), out.copy())
+        else:
+            assert np.array_equal(idx, first[t][0])
+            assert np.array_equal(out, first[t][1])  # deterministic, bit for bit
+
+
+def test_bf16_output_mode():
+    spec = synth.make_layer(56, 0, 1024, 2048, "bf16")
+    x = synth.make_tokens(56, 0, synth.ROLE_EVAL, 2, 1024, "bf16", rms_normalise=True)
+    t = float(np.quantile(np.abs(oracle.gate_activation(x, spec)), 0.5))
+    check_cats(spec, x, t, TOL_BF16, out_dtype=torch.bfloat16)
+
+
+# ------------------------------------------------------------------------------ full-size workloads
+
+@pytest.mark.parametrize("s", [0.5, 0.7, 0.9])
+def test_llama2_7b_batch1(s):
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=512)
+    t = oracle.calibrate_global(xc, spec, s)
+    layer = dev_layer(spec)
+    for b in range(2):
+        err, dens, _ = check_cats(spec, x[b:b + 1], t, TOL_BF16_F32OUT, layer=layer)
+        assert abs((1 - dens) - s) < 0.05
+
+
+def test_llama3_8b_union_batch4_and_16():
+    spec = synth.llama3_8b_stack_layer(0)
+    x = synth.make_tokens(3, 0, synth.ROLE_EVAL, 16, 4096, "bf16", rms_normalise=True)
+    t = float(np.quantile(np.abs(oracle.gate_activation(x, spec)), 0.5))
+    layer = dev_layer(spec)
+    err4, dens4, out4 = check_cats(spec, x[:4], t, TOL_BF16_F32OUT, layer=layer)
+    assert 0.85 < dens4 < 0.99
+    err16, dens16, out16 = check_cats(spec, x, t, TOL_BF16_F32OUT, layer=layer)
+    assert dens16 > 0.99
+    assert oracle.rel_l2(out16[:4], out4) <= TOL_BF16_F32OUT
+
+
+def test_llama3_70b_batch1_sampled():
+    spec, x, _ = synth.llama3_70b_swiglu(n_eval=1, n_calib=1)
+    a = np.abs(oracle.gate_activation(x, spec))
+    t = float(np.quantile(a, 0.9))
+    check_cats(spec, x, t, TOL_BF16_F32OUT)
+
+
+def test_llama3_70b_dense_verify_chunk():
+    spec, x, _ = synth.llama3_70b_swiglu(n_eval=16, n_calib=1)
+    out = run_dense(dev_layer(spec), x)
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16
