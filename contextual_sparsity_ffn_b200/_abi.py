@@ -58,6 +58,7 @@ SIGNATURES = {
     "csffn_kth_smallest": (_I, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _Z, _P]),
     "csffn_rmsnorm_bf16": (_I, [_P, _I, _I, _F, _P, _P]),
     "csffn_selftest_timeout": (_I, [_P, _Z, _I, _P]),
+    "csffn_sparse_ffn_forward_static": (_I, [_L, _P, _I, _P, _P, _P, _P, _I, _P]),
 }
 
 _lib = None

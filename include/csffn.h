@@ -9,7 +9,8 @@
  *    u_rt, v_r, values, ws is a DEVICE pointer owned by the caller.  The library
  *    keeps no pointer after the call returns and allocates no device memory on
  *    any path: scratch space comes from a caller workspace (`ws`) whose size is
- *    queried up front.
+ *    queried up front (csffn_sparse_ffn_forward_static instead uses one fixed
+ *    library-owned device array, see its comment).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous on that stream; nothing synchronises except
  *    csffn_check_status.  Index counts (`count`, `cand_count`) stay in device
@@ -197,6 +198,29 @@ csffn_status csffn_rmsnorm_bf16(const float* h, int B, int d, float eps, void* x
  * error word and returns; csffn_check_status then reports it.  The context stays
  * usable.  Run csffn_workspace_init afterwards. */
 csffn_status csffn_selftest_timeout(void* ws, size_t ws_bytes, int spin_limit, void* stream);
+
+/* Allocation-free variant of csffn_sparse_ffn_forward.  The pages have no counterpart: this is a
+ * deployment convenience of this library.
+ *   For callers that cannot allocate device memory at all, and so cannot create the workspace the
+ *   other entry points take: custom operators or plugins hosted by a framework that owns every
+ *   device allocation, and latency-critical loops that must not allocate after start-up.  The
+ *   caller still owns x, idx, count, a_val and out; the scratch of the gathered up/down projection
+ *   is a library-owned device array of CSFFN_STATIC_SCRATCH_BYTES, held by every GPU that loads
+ *   the library until the process exits.
+ *   Computes exactly what csffn_sparse_ffn_forward computes, with the same kernels.
+ *   Size limit: B*h*4 + 64*B*d*4 + 512 bytes (each term rounded up to 256) must fit in
+ *   CSFFN_STATIC_SCRATCH_BYTES, e.g. B <= 4 at d = 4096 and B <= 2 at d = 8192; larger calls
+ *   return CSFFN_ERR_UNSUPPORTED_SHAPE and launch nothing.
+ *   All calls share the one array: calls that overlap on the GPU (other streams, other host
+ *   threads) race, so order them on one stream.  The reduction counters are cleared on `stream`
+ *   before each launch; the rest of the array is fully rewritten before it is read.
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress with
+ *   that device current); make that first call before any stream capture that includes it.
+ *   Other arguments, layouts and errors as csffn_sparse_ffn_forward. */
+#define CSFFN_STATIC_SCRATCH_BYTES (8u << 20)
+csffn_status csffn_sparse_ffn_forward_static(const csffn_layer* layer, const void* x, int B,
+                                             const int32_t* idx, const int32_t* count, const float* a_val,
+                                             void* out, int out_mode, void* stream);
 
 #ifdef __cplusplus
 }
