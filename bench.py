@@ -53,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--sparsity", type=float, default=0.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-detail", action="store_true", help="skip the 70%/90%/dense detail runs")
+    ap.add_argument("--rotate", type=int, default=8,
+                    help="distinct layer weight sets the steps rotate over (8 keeps every step out of L2; "
+                         "1 only for profiler captures, which flush caches themselves)")
     return ap.parse_args(argv)
 
 
@@ -185,7 +188,7 @@ def profiled_traffic():
 # ---------------------------------------------------------------------------------- csffn arm
 
 def build_workload(torch, cs, synth, sparsities):
-    """8 rotation layers on the device, their thresholds per sparsity, and seeded tokens."""
+    """N_ROT rotation layers on the device, their thresholds per sparsity, and seeded tokens."""
     layers, thresholds = [], {s: [] for s in sparsities}
     for li in range(N_ROT):
         spec, _, xc = synth.llama2_7b_swiglu(li, n_eval=1, n_calib=512)
@@ -500,7 +503,9 @@ def reference_arm(args, world, rank):
 
 
 def main(argv=None) -> int:
+    global N_ROT
     args = parse_args(argv)
+    N_ROT = max(1, args.rotate)
     world, rank, local = dist_env()
     if args.impl == "reference":
         res, rank = reference_arm(args, world, rank)

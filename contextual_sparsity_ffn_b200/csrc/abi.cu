@@ -152,7 +152,7 @@ csffn_status csffn_gate_mask(const csffn_layer* layer, const void* x, int B, flo
   a.ctl = at<Control>(ws, L.ctl) + kCtlGate;
   a.status = at<uint64_t>(ws, L.status) + (size_t)kCtlGate * L.max_chunks;
   a.err = at<uint32_t>(ws, L.err);
-  return cuda_status(launch_gate_compact(a, layer->wdtype, false, kModeCats, as_stream(stream)));
+  return cuda_status(launch_gate(a, layer->wdtype, false, kModeCats, as_stream(stream)));
 }
 
 csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, int B,
@@ -182,7 +182,8 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
   u.count = count;
   u.a_val = a_val;
   u.v = at<float>(ws, L.vbuf);
-  cudaError_t e = launch_up_gather(u, layer->wdtype, s);
+  u.err = at<uint32_t>(ws, L.err);
+  cudaError_t e = launch_up(u, layer->wdtype, s);
   if (e != cudaSuccess) return CSFFN_ERR_CUDA;
 
   DownArgs dn{};
@@ -198,7 +199,8 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
   dn.slice_ctr = at<uint32_t>(ws, L.slice_ctr);
   dn.out = out;
   dn.out_mode = out_mode;
-  return cuda_status(launch_down_gather(dn, layer->wdtype, s));
+  dn.err = at<uint32_t>(ws, L.err);
+  return cuda_status(launch_down(dn, layer->wdtype, s));
 }
 
 csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,
@@ -248,7 +250,8 @@ csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, in
   dn.slice_ctr = at<uint32_t>(ws, L.slice_ctr) + kMaxSlices;
   dn.out = out;
   dn.out_mode = out_mode;
-  return cuda_status(launch_down_gather(dn, layer->wdtype, s));
+  dn.err = at<uint32_t>(ws, L.err);
+  return cuda_status(launch_down(dn, layer->wdtype, s));
 }
 
 csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int B, int rank,
@@ -298,7 +301,7 @@ csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int 
   a.ctl = at<Control>(ws, L.ctl) + kCtlPred;
   a.status = at<uint64_t>(ws, L.status) + (size_t)kCtlPred * L.max_chunks;
   a.err = at<uint32_t>(ws, L.err);
-  return cuda_status(launch_gate_compact(a, layer->wdtype, layer->wdtype == CSFFN_BF16, kModePred, s));
+  return cuda_status(launch_gate(a, layer->wdtype, layer->wdtype == CSFFN_BF16, kModePred, s));
 }
 
 // Calibration workspace: [header 512 B, error word at the decode layout's offset][kth state]

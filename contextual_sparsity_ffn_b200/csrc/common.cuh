@@ -49,7 +49,7 @@ struct WsLayout {
 
 constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   WsLayout L;
@@ -181,6 +181,69 @@ __device__ __forceinline__ bool bounded_wait(const uint64_t* p, uint32_t limit, 
     }
     __nanosleep(128);
   }
+}
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_now() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Decoupled look-back for chunk c, run by one full warp (all 32 lanes call it).
+//
+// Publishes the chunk's aggregate `agg`, then reads the status words of 32 predecessors at once
+// (lane l reads chunk base-l; positions before chunk 0 count as an inclusive prefix of 0).  As
+// soon as every predecessor up to the nearest inclusive prefix is published in this epoch, it sums
+// them and stops; if all 32 are published and none is inclusive, it adds the window's aggregates
+// and moves 32 chunks further back.  Publishes the chunk's inclusive prefix and returns the
+// exclusive one (the same in every lane).  A window that stays unusable for a second records
+// kDevErrTimeout in *err and ends the walk early (the caller keeps every write in bounds).
+__device__ __forceinline__ uint32_t warp_lookback(uint64_t* status, int c, uint32_t epoch, uint32_t agg,
+                                                  uint32_t* err, int lane) {
+  if (c == 0) {
+    if (lane == 0) st_release(&status[0], status_word(epoch, kFlagInclusive, agg));
+    return 0;
+  }
+  if (lane == 0) st_release(&status[c], status_word(epoch, kFlagAggregate, agg));
+  uint32_t prefix = 0;
+  uint64_t t0 = 0;
+  bool started = false;
+  for (int base = c - 1;;) {
+    const int j = base - lane;
+    const uint64_t s = j >= 0 ? ld_acquire(&status[j]) : status_word(epoch, kFlagInclusive, 0);
+    const bool ready = (uint32_t)(s >> 32) == epoch && ((s >> 30) & 3u) != 0;
+    const uint32_t ready_m = __ballot_sync(0xffffffffu, ready);
+    const uint32_t incl_m = __ballot_sync(0xffffffffu, ready && ((s >> 30) & 3u) == kFlagInclusive);
+    const int first_wait = ready_m == 0xffffffffu ? kWarp : __ffs(~ready_m) - 1;
+    const int first_incl = incl_m ? __ffs(incl_m) - 1 : kWarp;
+    const uint32_t val = (uint32_t)(s & 0x3FFFFFFFu);
+    if (first_incl < first_wait) {  // everything up to the nearest inclusive prefix is known
+      prefix += warp_sum_u32(lane <= first_incl ? val : 0u);
+      break;
+    }
+    if (first_wait == kWarp) {  // a full window of aggregates: add it and look further back
+      prefix += warp_sum_u32(val);
+      base -= kWarp;
+      started = false;
+      continue;
+    }
+    if (!started) {
+      t0 = globaltimer_now();
+      started = true;
+    } else if (globaltimer_now() - t0 > 1000000000ull) {
+      if (lane == 0) atomicOr(err, kDevErrTimeout);
+      break;
+    }
+    __nanosleep(32);
+  }
+  if (lane == 0) st_release(&status[c], status_word(epoch, kFlagInclusive, prefix + agg));
+  return prefix;
 }
 
 }  // namespace csffn

@@ -49,11 +49,13 @@ static cudaError_t allow_smem(K kern, size_t smem) {
 // ------------------------------------------------------------------------------------------
 // Up projection over the compacted active list: v[b, j] = a_val[b, j] * (x_b . W_up[idx[j]])
 // ------------------------------------------------------------------------------------------
+// One row per warp at a time with GemvUnroll vectors in flight per lane, four CTAs per SM: many
+// independent row streams keep HBM busy (a gathered row cannot be fetched as one large block).
 template <typename WT, int NB>
-__global__ void __launch_bounds__(kThreads) up_gather_kernel(const UpArgs p) {
+__global__ void __launch_bounds__(kThreads, 4) up_gather_kernel(const UpArgs p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   WT* xs = reinterpret_cast<WT*>(smem_raw);
-  constexpr int R = 2;
+  constexpr int R = 1;
   constexpr int U = GemvUnroll<NB>::value;
   const int lane = threadIdx.x & 31;
   stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), p.B, p.d);
@@ -319,7 +321,7 @@ static cudaError_t up_t(const UpArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)NB * a.d * sizeof(WT);
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  const int grid = grid_for(kern, smem, (a.h + 1) / 2);
+  const int grid = grid_for(kern, smem, a.h);
   kern<<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
@@ -341,7 +343,8 @@ static cudaError_t down_t(const DownArgs& a, cudaStream_t s) {
   constexpr int SW = kWarp * Vec<WT>::N;
   const int slices = (a.d + SW - 1) / SW;
   const int occ = occupancy(kern, kThreads, 0);
-  int ry = (sm_count() * occ + slices - 1) / slices;
+  int ry = (sm_count() * occ) / slices;  // one wave: every CTA resident at once
+  if (ry < 1) ry = 1;
   if (ry > kMaxRowRanges) ry = kMaxRowRanges;
   const int max_rows = a.count ? a.h : a.n_host;
   if (ry > max_rows) ry = max_rows > 0 ? max_rows : 1;

@@ -112,26 +112,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_compact_kernel(const GateAr
       const bool keep = lane < kChunkRows && s_keep[lane] != 0u;
       const uint32_t mask = __ballot_sync(0xffffffffu, keep);
       const uint32_t agg = __popc(mask);
-      uint32_t prefix = 0;
-      if (lane == 0) {
-        if (c == 0) {
-          st_release(&p.status[0], status_word(epoch, kFlagInclusive, agg));
-        } else {
-          st_release(&p.status[c], status_word(epoch, kFlagAggregate, agg));
-          // Walk back over predecessors: add aggregates until an inclusive prefix is found.
-          for (int j = c - 1; j >= 0; --j) {
-            uint64_t s = 0;
-            const bool ok = bounded_wait(
-                &p.status[j], kSpinLimit, p.err,
-                [epoch](uint64_t v) { return (uint32_t)(v >> 32) == epoch && ((v >> 30) & 3u) != 0; }, &s);
-            if (!ok) break;  // predecessor never published: recorded in the error word
-            prefix += (uint32_t)(s & 0x3FFFFFFFu);
-            if (((s >> 30) & 3u) == kFlagInclusive) break;
-          }
-          st_release(&p.status[c], status_word(epoch, kFlagInclusive, prefix + agg));
-        }
-      }
-      prefix = __shfl_sync(0xffffffffu, prefix, 0);
+      const uint32_t prefix = warp_lookback(p.status, c, epoch, agg, p.err, lane);
       if (keep) {
         const uint32_t pos = prefix + __popc(mask & ((1u << lane) - 1u));
         if (pos < (uint32_t)p.h) {

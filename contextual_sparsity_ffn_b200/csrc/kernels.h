@@ -32,6 +32,15 @@ struct GateArgs {
   uint32_t* err;
 };
 cudaError_t launch_gate_compact(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
+// Same computation, warp-specialised and fed by bulk copies (gate_tma.cu); needs a ring of at least
+// four 2-row slots beside the staged tokens in shared memory.
+bool gate_tma_supported(int K, int B, int wdtype, bool x_f32);
+cudaError_t launch_gate_tma(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
+// Picks the bulk-copy kernel when the shape allows it, else the register-streaming one.
+inline cudaError_t launch_gate(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s) {
+  return gate_tma_supported(a.K, a.B, wdtype, x_f32) ? launch_gate_tma(a, wdtype, x_f32, mode, s)
+                                                     : launch_gate_compact(a, wdtype, x_f32, mode, s);
+}
 
 // v[b*h + j] = a_val[b*h + j] * (x_b . W_up[idx[j]]) for j < *count.
 struct UpArgs {
@@ -42,8 +51,10 @@ struct UpArgs {
   const int32_t* count;
   const float* a_val;
   float* v;
+  uint32_t* err;  // device error word (for kernels with bounded waits)
 };
 cudaError_t launch_up_gather(const UpArgs& a, int wdtype, cudaStream_t s);
+inline cudaError_t launch_up(const UpArgs& a, int wdtype, cudaStream_t s) { return launch_up_gather(a, wdtype, s); }
 
 // v[b*h + i] = act(x_b . W_gate[i] + beta_i) * (x_b . W_up[i]) for all i < h.
 struct DenseGateUpArgs {
@@ -69,8 +80,10 @@ struct DownArgs {
   uint32_t* slice_ctr;    // [slices]
   void* out;
   int out_mode;
+  uint32_t* err;  // device error word (for kernels with bounded waits)
 };
 cudaError_t launch_down_gather(const DownArgs& a, int wdtype, cudaStream_t s);
+inline cudaError_t launch_down(const DownArgs& a, int wdtype, cudaStream_t s) { return launch_down_gather(a, wdtype, s); }
 
 // y[b*rank + k] = x_b . U_r^T[k]  (plain GEMV, fp32 out)
 struct RowGemvArgs {
