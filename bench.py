@@ -6,8 +6,10 @@ accumulation, batch-1 decode, CATS threshold calibrated by csffn_calibrate_thres
 on 512 seeded calibration vectors at 50% target sparsity (70% and 90% and the dense
 path of the same library are measured too and reported under "detail").
 
-A step is one CATS decode of one layer: csffn_gate_mask (gate GEMV + SiLU + threshold
-+ compaction) then csffn_sparse_ffn_forward (gathered up and down projections).  The
+A step is one CATS decode of one layer through csffn_cats_ffn_forward: gate GEMV + SiLU
++ threshold + gathered up projection, a grid barrier, then the gathered down projection
+and the compaction of the active list, in one kernel launch.  The two-call path
+(csffn_gate_mask then csffn_sparse_ffn_forward, three kernels) is reported under "detail".  The
 timed steps rotate over 8 distinct layer weight sets (2.2 GB, many times the 126 MB L2)
 so no step reads weights that an earlier step left in L2.  K steps are captured in one
 CUDA graph and timed with CUDA events on the capture stream.
@@ -41,6 +43,9 @@ FALLBACK_HBM_GBS = 6650.0
 D, H = 4096, 11008
 N_ROT = 8
 N_TOKENS = 64
+# Headline path: the two-call path (csffn_gate_mask + csffn_sparse_ffn_forward) measures faster
+# than the one-launch csffn_cats_ffn_forward on this workload; both are reported.
+HEADLINE_TWO_CALL = True
 PROFILE_SUMMARY = os.path.join(HERE, "profiles", "gate_mask_llama2_7b_b1.md")
 
 
@@ -232,16 +237,23 @@ def csffn_arm(args, world, rank, local):
     stream = torch.cuda.Stream()
     K, W = args.steps, args.warmup
 
-    def sparse_step(s, gate_events=None):
+    def sparse_step(s, events=None, two_call=HEADLINE_TWO_CALL):
+        """One decode step on layer k % N_ROT: the one-launch csffn_cats_ffn_forward, or the
+        two-call path csffn_gate_mask + csffn_sparse_ffn_forward."""
         def f(k):
             li = k % N_ROT
             x = xs[k % N_TOKENS: k % N_TOKENS + 1]
-            if gate_events is not None:
-                gate_events[k][0].record()
-            cs.gate_mask(layers[li], x, thr[s][li], buf.idx, buf.count, buf.a_val, buf.ws)
-            if gate_events is not None:
-                gate_events[k][1].record()
-            cs.sparse_ffn_forward(layers[li], x, buf.idx, buf.count, buf.a_val, out, buf.ws)
+            if events is not None:
+                events[k][0].record()
+            if two_call:
+                cs.gate_mask(layers[li], x, thr[s][li], buf.idx, buf.count, buf.a_val, buf.ws)
+                if events is not None:
+                    events[k][1].record()
+                cs.sparse_ffn_forward(layers[li], x, buf.idx, buf.count, buf.a_val, out, buf.ws)
+            else:
+                cs.cats_ffn_forward(layers[li], x, thr[s][li], buf.idx, buf.count, buf.a_val, out, buf.ws)
+                if events is not None:
+                    events[k][1].record()
         return f
 
     def dense_step(k):
@@ -290,8 +302,8 @@ def csffn_arm(args, world, rank, local):
     if gate_in_graph:
         gate_ms = [a.elapsed_time(b) for a, b in gate_ev]
     else:
-        gate_ms = time_gate_eager(torch, cs, layers, thr[args.sparsity], xs, buf, stream, K)
-    gate_avg_us = 1000.0 * float(np.mean(gate_ms))
+        gate_ms = time_step_eager(torch, cs, layers, thr[args.sparsity], xs, buf, out, stream, K)
+    kern_avg_us = 1000.0 * float(np.mean(gate_ms))
 
     # active rows actually read per step (deterministic; recomputed eagerly)
     counts = []
@@ -310,11 +322,26 @@ def csffn_arm(args, world, rank, local):
     us = whole_job_us_per_layer(ms_max, K, world)
     us_gpu = ms_max * 1000.0 / K  # one GPU's time per layer-step
     gbs = step_bytes(n_act) / (us_gpu * 1e-6) / 1e9  # per GPU
-    gate_bytes = 2.0 * H * D + 2 * D + 8.0 * n_act + 4.0 * n_act
-    gate_gbs = gate_bytes / (gate_avg_us * 1e-6) / 1e9
+    if HEADLINE_TWO_CALL:
+        # dominant kernel: the gate (reads all of W_gate); events bracket csffn_gate_mask
+        kern_name = "gate_stream_kernel (csffn_gate_mask)"
+        kern_bytes = 2.0 * H * D + 2 * D + 8.0 * n_act
+    else:
+        kern_name = "cats_fused_kernel (csffn_cats_ffn_forward)"
+        kern_bytes = step_bytes(n_act)  # the whole step is one kernel launch
+    kern_gbs = kern_bytes / (kern_avg_us * 1e-6) / 1e9
 
     detail = {}
     if not args.no_detail:
+        other = not HEADLINE_TWO_CALL
+        g = run_graph_steps(torch, sparse_step(args.sparsity, two_call=other), K, W, stream)
+        t2 = max_over_ranks(time_graph(g, warm_replays), world, dev)
+        u2 = whole_job_us_per_layer(t2, K, world)
+        detail[f"{'two_call' if other else 'one_launch'}_{int(round(args.sparsity * 100))}"] = {
+            "path": "csffn_gate_mask + csffn_sparse_ffn_forward (3 kernels)" if other
+                    else "csffn_cats_ffn_forward (1 kernel)", "us_per_layer": round(u2, 3),
+            "achieved_gbs": round(step_bytes(n_act) / (u2 * 1e-6) / 1e9, 1)}
+        del g
         for s in sparsities[1:]:
             g = run_graph_steps(torch, sparse_step(s), K, W, stream)
             t = time_graph(g, warm_replays)
@@ -366,15 +393,16 @@ def csffn_arm(args, world, rank, local):
         "achieved_gbs": round(gbs, 1),
         "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
         f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4),
-        "roofline": {"bound": "hbm", "kernel": "gate_compact_kernel (csffn_gate_mask)",
-                     "achieved": round(gate_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "peak_source": f"{peak_kind} copy bandwidth", "frac": round(gate_gbs / peak, 4),
-                     "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": round(gate_bytes),
-                     "avg_launch_us": round(gate_avg_us, 3),
+        "roofline": {"bound": "hbm", "kernel": kern_name,
+                     "achieved": round(kern_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "peak_source": f"{peak_kind} copy bandwidth", "frac": round(kern_gbs / peak, 4),
+                     "frac_of_8tbs": round(kern_gbs / NOMINAL_HBM_GBS, 4),
+                     "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": round(kern_bytes),
+                     "avg_launch_us": round(kern_avg_us, 3),
                      "timing": "events around each launch inside the timed graph" if gate_in_graph
                                else "events around eager launches"},
         "e2e": e2e,
-        "gpu_launches": 3 * K,
+        "gpu_launches": (3 if HEADLINE_TWO_CALL else 1) * K,
         "clocks": clocks,
     }
     if detail:
@@ -384,16 +412,21 @@ def csffn_arm(args, world, rank, local):
     return result, rank
 
 
-def time_gate_eager(torch, cs, layers, thr, xs, buf, stream, K):
+def time_step_eager(torch, cs, layers, thr, xs, buf, out_t, stream, K):
     out = []
     with torch.cuda.stream(stream):
         for k in range(K):
             li = k % N_ROT
+            x = xs[k % N_TOKENS: k % N_TOKENS + 1]
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            cs.gate_mask(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], thr[li], buf.idx, buf.count,
-                         buf.a_val, buf.ws)
+            if HEADLINE_TWO_CALL:
+                cs.gate_mask(layers[li], x, thr[li], buf.idx, buf.count, buf.a_val, buf.ws)
+            else:
+                cs.cats_ffn_forward(layers[li], x, thr[li], buf.idx, buf.count, buf.a_val, out_t, buf.ws)
             b.record()
+            if HEADLINE_TWO_CALL:
+                cs.sparse_ffn_forward(layers[li], x, buf.idx, buf.count, buf.a_val, out_t, buf.ws)
             out.append((a, b))
     torch.cuda.synchronize()
     return [a.elapsed_time(b) for a, b in out]

@@ -148,6 +148,17 @@ def sparse_ffn_forward(layer: FFNLayer, x: torch.Tensor, idx: torch.Tensor, coun
           "csffn_sparse_ffn_forward")
 
 
+def cats_ffn_forward(layer: FFNLayer, x: torch.Tensor, t: float, idx: torch.Tensor, count: torch.Tensor,
+                     a_val: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, out_mode: Optional[int] = None,
+                     stream=None) -> None:
+    B = x.shape[0] if x.dim() == 2 else 1
+    if out_mode is None:
+        out_mode = _abi.OUT_BF16 if out.dtype == torch.bfloat16 else _abi.OUT_F32
+    check(load().csffn_cats_ffn_forward(layer.ref(), _ptr(x), B, float(t), _ptr(idx), _ptr(count), _ptr(a_val),
+                                        _ptr(out), out_mode, _ptr(ws), _nbytes(ws), _stream(stream)),
+          "csffn_cats_ffn_forward")
+
+
 def dense_ffn_forward(layer: FFNLayer, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
                       out_mode: Optional[int] = None, stream=None) -> None:
     B = x.shape[0] if x.dim() == 2 else 1
@@ -229,7 +240,11 @@ class DecodeBuffers:
 
 
 def cats_decode(layer: FFNLayer, x: torch.Tensor, t: float, out: torch.Tensor, buf: DecodeBuffers,
-                out_mode: Optional[int] = None, stream=None) -> None:
-    """One CATS sparse FFN step: csffn_gate_mask then csffn_sparse_ffn_forward."""
+                out_mode: Optional[int] = None, stream=None, one_launch: bool = False) -> None:
+    """One CATS sparse FFN step: csffn_gate_mask then csffn_sparse_ffn_forward, or with
+    one_launch the single-kernel csffn_cats_ffn_forward (same outputs)."""
+    if one_launch:
+        cats_ffn_forward(layer, x, t, buf.idx, buf.count, buf.a_val, out, buf.ws, out_mode=out_mode, stream=stream)
+        return
     gate_mask(layer, x, t, buf.idx, buf.count, buf.a_val, buf.ws, stream=stream)
     sparse_ffn_forward(layer, x, buf.idx, buf.count, buf.a_val, out, buf.ws, out_mode=out_mode, stream=stream)

@@ -203,6 +203,54 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
   return cuda_status(launch_down(dn, layer->wdtype, s));
 }
 
+csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
+                                    int32_t* idx, int32_t* count, float* a_val,
+                                    void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
+  csffn_status st = check_layer_shape(layer);
+  if (st != CSFFN_OK) return st;
+  if (B < 0 || B > CSFFN_MAX_BATCH) return CSFFN_ERR_INVALID_ARG;
+  if (out_mode != CSFFN_OUT_BF16 && out_mode != CSFFN_OUT_F32 && out_mode != CSFFN_OUT_F32_ACCUMULATE)
+    return CSFFN_ERR_INVALID_ARG;
+  if (!count) return CSFFN_ERR_INVALID_ARG;
+  if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
+  if (!cats_fused_supported(layer->d, B, layer->wdtype)) {
+    st = csffn_gate_mask(layer, x, B, t, nullptr, nullptr, idx, count, a_val, ws, ws_bytes, stream);
+    if (st != CSFFN_OK) return st;
+    return csffn_sparse_ffn_forward(layer, x, B, idx, count, a_val, out, out_mode, ws, ws_bytes, stream);
+  }
+  if (!x || !idx || !a_val || !out || std::isnan(t)) return CSFFN_ERR_INVALID_ARG;
+  if ((st = check_weights(layer, true, true, true)) != CSFFN_OK) return st;
+  if (!aligned16(x) || !aligned16(out)) return CSFFN_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(layer->d, layer->h, B, 0);
+  if ((st = check_ws(ws, ws_bytes, L.ybuf)) != CSFFN_OK) return st;
+  FusedArgs a{};
+  a.W_gate = layer->w_gate;
+  a.W_up = layer->w_up;
+  a.W_down_t = layer->w_down_t;
+  a.x = x;
+  a.d = layer->d;
+  a.h = layer->h;
+  a.B = B;
+  a.bias = layer->gate_bias;
+  a.t = t;
+  a.act = layer->act;
+  a.v = at<float>(ws, L.vbuf);
+  a.afull = at<float>(ws, L.afull);
+  a.flags = at<uint8_t>(ws, L.flags);
+  a.partial = at<float>(ws, L.partial);
+  a.slice_ctr = at<uint32_t>(ws, L.slice_ctr);
+  a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
+  a.range_cnt = at<uint32_t>(ws, L.range_cnt);
+  a.tickets = at<uint32_t>(ws, L.tickets);
+  a.err = at<uint32_t>(ws, L.err);
+  a.idx = idx;
+  a.count = count;
+  a.a_val = a_val;
+  a.out = out;
+  a.out_mode = out_mode;
+  return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
+}
+
 csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,
                                      void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
   csffn_status st = check_layer_shape(layer);

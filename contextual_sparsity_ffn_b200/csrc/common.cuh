@@ -29,6 +29,7 @@ struct Control {           // one per compaction user, 64 bytes apart
 
 constexpr int kCtlGate = 0;     // csffn_gate_mask
 constexpr int kCtlPred = 1;     // csffn_predict_lowrank
+constexpr int kCtlFused = 2;    // csffn_cats_ffn_forward (tile and exit counters)
 constexpr int kNumCtl = 4;
 constexpr int kMaxSlices = 128;  // column slices of the down projection (d / slice width)
 constexpr int kMaxRowRanges = 64;
@@ -38,9 +39,13 @@ struct WsLayout {
   size_t ctl;        // Control[kNumCtl]
   size_t err;        // uint32 error word (+ pad)
   size_t slice_ctr;  // uint32 [kSliceUsers][kMaxSlices]
+  size_t range_cnt;  // uint32 [2][kMaxRowRanges]       kept rows per neuron range (fused path)
+  size_t tickets;    // uint32 [64][32]                 row-ticket counters, 128 B apart (fused path)
   size_t status;     // uint64 [kNumCtl][max_chunks]   look-back status words
   size_t control_end;
   size_t vbuf;       // fp32 [max_batch][h]            v = a * u (sparse) or act(z)*u (dense)
+  size_t afull;      // fp32 [max_batch][h]            per-neuron kept activations (fused path)
+  size_t flags;      // uint8 [h]                      per-neuron keep flags (fused path)
   size_t partial;    // fp32 [kMaxRowRanges][max_batch][d]
   size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
   size_t total;
@@ -57,12 +62,19 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   L.ctl = o;        o += sizeof(Control) * kNumCtl;
   L.err = o;        o += 64;
   L.slice_ctr = o;  o += sizeof(uint32_t) * kSliceUsers * kMaxSlices;
+  L.range_cnt = o;  o += sizeof(uint32_t) * 2 * kMaxRowRanges;
+  o = align_up(o, 128);
+  L.tickets = o;    o += sizeof(uint32_t) * 64 * 32;
   o = align_up(o, 256);
   L.max_chunks = (h + kChunkRows - 1) / kChunkRows;
   L.status = o;     o += sizeof(uint64_t) * (size_t)kNumCtl * L.max_chunks;
   o = align_up(o, 256);
   L.control_end = o;
   L.vbuf = o;       o += sizeof(float) * (size_t)max_batch * h;
+  o = align_up(o, 256);
+  L.afull = o;      o += sizeof(float) * (size_t)max_batch * h;
+  o = align_up(o, 256);
+  L.flags = o;      o += align_up((size_t)h, 16);
   o = align_up(o, 256);
   L.partial = o;    o += sizeof(float) * (size_t)kMaxRowRanges * max_batch * d;
   o = align_up(o, 256);
@@ -88,6 +100,19 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
       : "l"(p));
   return r;
 }
+
+// Asynchronous 16-byte global -> shared copy by this thread (cp.async, cached in L2 only).  The
+// data is this thread's own: it waits for it with cp_async_wait<N> and nothing else is needed.
+// `after` is a value the copy must not be issued before (a register dependency that orders the
+// copy after the thread's earlier reads of the same shared memory).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, uint32_t after) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(src), "r"(after)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -125,6 +150,12 @@ __device__ __forceinline__ void load_x(const float* p, float (&f)[N]) {
   }
 }
 
+// 16 bytes of token values (same element type as the weights) -> floats.
+template <typename T>
+__device__ __forceinline__ void unpack_x(const uint4& v, float (&f)[Vec<T>::N]) {
+  unpack(v, f);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -137,20 +168,18 @@ __device__ __forceinline__ float gate_act(float z, int act) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Acquire/release accesses for cross-CTA status words
+// Cross-CTA status words.  A status word carries only a count that the reader adds up; no other
+// data written by the publishing CTA is read through it inside the kernel (outputs are consumed
+// by later launches), so single-copy-atomic relaxed accesses at GPU scope suffice and the
+// publishing thread pays no fence.
 // ------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t ld_acquire(const uint64_t* p) {
+__device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
   uint64_t v;
-  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void st_release(uint64_t* p, uint64_t v) {
-  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void st_status(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // Look-back status word: [epoch:32 | flag:2 | value:30].
@@ -163,14 +192,14 @@ __device__ __forceinline__ uint64_t status_word(uint32_t epoch, uint64_t flag, u
 // far beyond any wait on a CTA that is running.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
-// Bounded wait on a 64-bit status word: polls *p (acquire) until ready(value) holds or `limit`
+// Bounded wait on a 64-bit status word: polls *p until ready(value) holds or `limit`
 // polls have failed.  On success returns true with the word in *out; on give-up records
 // kDevErrTimeout in *err and returns false.  Every device-side wait in the library uses this.
 template <typename Ready>
 __device__ __forceinline__ bool bounded_wait(const uint64_t* p, uint32_t limit, uint32_t* err,
                                              Ready ready, uint64_t* out) {
   for (uint32_t spins = 0;; ++spins) {
-    const uint64_t v = ld_acquire(p);
+    const uint64_t v = ld_status(p);
     if (ready(v)) {
       *out = v;
       return true;
@@ -204,19 +233,21 @@ __device__ __forceinline__ uint64_t globaltimer_now() {
 // and moves 32 chunks further back.  Publishes the chunk's inclusive prefix and returns the
 // exclusive one (the same in every lane).  A window that stays unusable for a second records
 // kDevErrTimeout in *err and ends the walk early (the caller keeps every write in bounds).
+// With agg_published the caller has already published the chunk's aggregate (chunk 0: its
+// inclusive prefix), so only the walk and the inclusive publication remain.
 __device__ __forceinline__ uint32_t warp_lookback(uint64_t* status, int c, uint32_t epoch, uint32_t agg,
-                                                  uint32_t* err, int lane) {
+                                                  uint32_t* err, int lane, bool agg_published = false) {
   if (c == 0) {
-    if (lane == 0) st_release(&status[0], status_word(epoch, kFlagInclusive, agg));
+    if (lane == 0 && !agg_published) st_status(&status[0], status_word(epoch, kFlagInclusive, agg));
     return 0;
   }
-  if (lane == 0) st_release(&status[c], status_word(epoch, kFlagAggregate, agg));
+  if (lane == 0 && !agg_published) st_status(&status[c], status_word(epoch, kFlagAggregate, agg));
   uint32_t prefix = 0;
   uint64_t t0 = 0;
   bool started = false;
   for (int base = c - 1;;) {
     const int j = base - lane;
-    const uint64_t s = j >= 0 ? ld_acquire(&status[j]) : status_word(epoch, kFlagInclusive, 0);
+    const uint64_t s = j >= 0 ? ld_status(&status[j]) : status_word(epoch, kFlagInclusive, 0);
     const bool ready = (uint32_t)(s >> 32) == epoch && ((s >> 30) & 3u) != 0;
     const uint32_t ready_m = __ballot_sync(0xffffffffu, ready);
     const uint32_t incl_m = __ballot_sync(0xffffffffu, ready && ((s >> 30) & 3u) == kFlagInclusive);
@@ -242,7 +273,7 @@ __device__ __forceinline__ uint32_t warp_lookback(uint64_t* status, int c, uint3
     }
     __nanosleep(32);
   }
-  if (lane == 0) st_release(&status[c], status_word(epoch, kFlagInclusive, prefix + agg));
+  if (lane == 0) st_status(&status[c], status_word(epoch, kFlagInclusive, prefix + agg));
   return prefix;
 }
 

@@ -51,45 +51,74 @@ static cudaError_t allow_smem(K kern, size_t smem) {
 // ------------------------------------------------------------------------------------------
 // One row per warp at a time with GemvUnroll vectors in flight per lane, four CTAs per SM: many
 // independent row streams keep HBM busy (a gathered row cannot be fetched as one large block).
+// A warp's row indices and a_val values are fetched once, up front, one per lane.  The tokens are
+// staged in shared memory (measured faster than reading them through the read-only cache).
 template <typename WT, int NB>
 __global__ void __launch_bounds__(kThreads, 4) up_gather_kernel(const UpArgs p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  WT* xs = reinterpret_cast<WT*>(smem_raw);
-  constexpr int R = 1;
+  constexpr bool kStage = true;
+  constexpr int EPV = Vec<WT>::N;
   constexpr int U = GemvUnroll<NB>::value;
   const int lane = threadIdx.x & 31;
-  stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), p.B, p.d);
-  __syncthreads();
+  const WT* xs = reinterpret_cast<const WT*>(p.x);
+  if (kStage) {
+    stage_tokens<WT, NB>(reinterpret_cast<WT*>(smem_raw), reinterpret_cast<const WT*>(p.x), p.B, p.d);
+    __syncthreads();
+    xs = reinterpret_cast<const WT*>(smem_raw);
+  }
   const int n = min(max(*p.count, 0), p.h);
-  const int groups = (n + R - 1) / R;
   const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int GW = gridDim.x * kWarps;
   const WT* W = reinterpret_cast<const WT*>(p.W_up);
-  for (int g = gw; g < groups; g += GW) {
-    const WT* rp[R];
-    bool valid[R];
+  const int NV = p.d / EPV;
+  for (int j0 = gw; j0 < n; j0 += GW * kWarp) {
+    // rows j0 + k*GW for k = 0..31, one per lane: index and per-token a_val
+    const int my_j = j0 + lane * GW;
+    int my_row = my_j < n ? p.idx[my_j] : 0;
+    if ((unsigned)my_row >= (unsigned)p.h) my_row = 0;  // malformed index: stay in bounds
+    float my_a[NB];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int j = g * R + r;
-      valid[r] = j < n;
-      int row = valid[r] ? p.idx[j] : 0;
-      if ((unsigned)row >= (unsigned)p.h) row = 0;  // malformed index: stay in bounds
-      rp[r] = W + (size_t)row * p.d;
-    }
-    float acc[R][NB];
+    for (int b = 0; b < NB; ++b) my_a[b] = (my_j < n && b < p.B) ? p.a_val[(size_t)b * p.h + my_j] : 0.f;
+    const int cnt = __popc(__ballot_sync(0xffffffffu, my_j < n));
+    for (int k = 0; k < cnt; ++k) {
+      const WT* row = W + (size_t)__shfl_sync(0xffffffffu, my_row, k) * p.d;
+      float acc[NB];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+      for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      for (int v0 = lane; v0 < NV; v0 += kWarp * U) {
+        uint4 w[U];
 #pragma unroll
-      for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
-    rows_dot<WT, WT, NB, R, U>(rp, valid, xs, p.d, lane, acc);
-    warp_reduce_all<R, NB>(acc);
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * kWarp;
+          w[u] = v < NV ? ld_stream(row + (size_t)v * EPV) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (lane == r && valid[r]) {
-        const size_t j = (size_t)g * R + r;
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * kWarp;
+          if (v < NV) {
+            float wf[EPV];
+            unpack(w[u], wf);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              float xf[EPV];
+              if (kStage) {
+                load_x<EPV>(xs + (size_t)b * p.d + (size_t)v * EPV, xf);
+              } else {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xs + (size_t)b * p.d + (size_t)v * EPV));
+                unpack_x<WT>(xv, xf);
+              }
+#pragma unroll
+              for (int e = 0; e < EPV; ++e) acc[b] = fmaf(wf[e], xf[e], acc[b]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
+      if (lane == k) {
 #pragma unroll
         for (int b = 0; b < NB; ++b)
-          if (b < p.B) p.v[(size_t)b * p.h + j] = p.a_val[(size_t)b * p.h + j] * acc[r][b];
+          if (b < p.B) p.v[(size_t)b * p.h + my_j] = my_a[b] * acc[b];
       }
     }
   }
@@ -148,13 +177,17 @@ __global__ void __launch_bounds__(kThreads) dense_gate_up_kernel(const DenseGate
 // ------------------------------------------------------------------------------------------
 // Down projection over rows idx[0..n): out[b, :] = sum_j v[b, j] * W_down^T[idx[j], :]
 // ------------------------------------------------------------------------------------------
-template <int NB> struct DownUnroll { static constexpr int value = NB <= 2 ? 8 : (NB <= 4 ? 4 : 2); };
+// Rows per pipeline unit (one 16-byte vector per lane per row) and resident CTAs per SM the
+// register budget is capped for.
+template <int NB> struct DownUnroll { static constexpr int value = NB <= 2 ? 4 : 2; };
+template <int NB> struct DownMinBlocks { static constexpr int value = NB <= 2 ? 4 : (NB <= 4 ? 3 : 1); };
 
 template <typename WT, int NB>
-__global__ void __launch_bounds__(kThreads) down_gather_kernel(const DownArgs p) {
+__global__ void __launch_bounds__(kThreads, DownMinBlocks<NB>::value) down_gather_kernel(const DownArgs p) {
   constexpr int EPV = Vec<WT>::N;
   constexpr int SW = kWarp * EPV;  // columns per slice
   constexpr int U = DownUnroll<NB>::value;
+  static_assert(kWarp % U == 0, "units never straddle a 32-row batch");
   __shared__ float red[kWarps][SW];
   __shared__ bool s_last;
 
@@ -172,36 +205,73 @@ __global__ void __launch_bounds__(kThreads) down_gather_kernel(const DownArgs p)
 #pragma unroll
     for (int e = 0; e < EPV; ++e) acc[b][e] = 0.f;
 
-  // This warp's rows: jb + warp, jb + warp + 8, ...; fetched 32 at a time (one per lane).
-  for (int m0 = jb + warp; m0 < je; m0 += kWarps * kWarp) {
-    const int my_j = m0 + lane * kWarps;
-    const bool my_ok = my_j < je;
-    int my_row = my_ok ? (p.idx ? p.idx[my_j] : my_j) : 0;
-    if ((unsigned)my_row >= (unsigned)p.h) my_row = 0;  // malformed index: stay in bounds
-    float my_v[NB];
+  // This warp's rows: m-th row is jb + warp + 8m, m < M.  Row indices and v values come in
+  // batches of 32 (one per lane), the next batch fetched while the current one streams; the
+  // weight loads run as a double-buffered pipeline of U-row units.
+  const int M = je - jb - warp > 0 ? (je - jb - warp + kWarps - 1) / kWarps : 0;
+  auto fetch = [&](int batch, int& row, float (&v)[NB]) {
+    const int m = batch * kWarp + lane;
+    const int j = jb + warp + m * kWarps;
+    const bool ok = m < M;
+    row = ok ? (p.idx ? p.idx[j] : j) : 0;
+    if ((unsigned)row >= (unsigned)p.h) row = 0;  // malformed index: stay in bounds
 #pragma unroll
-    for (int b = 0; b < NB; ++b) my_v[b] = (my_ok && b < p.B) ? p.v[(size_t)b * p.h + my_j] : 0.f;
-    const int cnt = __popc(__ballot_sync(0xffffffffu, my_ok));
-    for (int q = 0; q < cnt; q += U) {
-      uint4 w[U];
+    for (int b = 0; b < NB; ++b) v[b] = (ok && b < p.B) ? p.v[(size_t)b * p.h + j] : 0.f;
+  };
+  int cur_row = 0, nxt_row = 0;
+  float cur_v[NB], nxt_v[NB];
+  fetch(0, cur_row, cur_v);
+  fetch(1, nxt_row, nxt_v);
+  const int units = (M + U - 1) / U;
+  constexpr int UPB = kWarp / U;  // units per batch
+  uint4 bufA[U], bufB[U];
+  auto load_unit = [&](int t, int cb, uint4 (&buf)[U]) {
+    const int from_next = (t / UPB) != cb;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int row = __shfl_sync(0xffffffffu, my_row, (q + u) & 31);
-        w[u] = (q + u < cnt && col_ok) ? ld_stream(Wd + (size_t)row * p.d + c0) : make_uint4(0u, 0u, 0u, 0u);
-      }
+    for (int u = 0; u < U; ++u) {
+      const int m = t * U + u;
+      const int src = m % kWarp;
+      const int r = __shfl_sync(0xffffffffu, from_next ? nxt_row : cur_row, src);
+      buf[u] = (m < M && col_ok) ? ld_stream(Wd + (size_t)r * p.d + c0) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto consume = [&](int t, const uint4 (&buf)[U]) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float wf[EPV];
-        unpack(w[u], wf);
+    for (int u = 0; u < U; ++u) {
+      const int m = t * U + u;
+      float wf[EPV];
+      unpack(buf[u], wf);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float vb = __shfl_sync(0xffffffffu, my_v[b], (q + u) & 31);
-          if (q + u < cnt) {
+      for (int b = 0; b < NB; ++b) {
+        const float vb = __shfl_sync(0xffffffffu, cur_v[b], m % kWarp);
+        if (m < M) {
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[b][e] = fmaf(vb, wf[e], acc[b][e]);
-          }
+          for (int e = 0; e < EPV; ++e) acc[b][e] = fmaf(vb, wf[e], acc[b][e]);
         }
       }
+    }
+  };
+  int cb = 0;  // batch held in cur_*
+  if (units > 0) load_unit(0, cb, bufA);
+  for (int t = 0; t < units; t += 2) {
+    if (t + 1 < units) load_unit(t + 1, cb, bufB);
+    consume(t, bufA);
+    if ((t + 1) % UPB == 0 && t + 1 < units) {  // unit t closed batch cb
+      ++cb;
+      cur_row = nxt_row;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) cur_v[b] = nxt_v[b];
+      fetch(cb + 1, nxt_row, nxt_v);
+    }
+    if (t + 1 >= units) break;
+    if (t + 2 < units) load_unit(t + 2, cb, bufA);
+    consume(t + 1, bufB);
+    if ((t + 2) % UPB == 0 && t + 2 < units) {  // unit t + 1 closed batch cb
+      ++cb;
+      cur_row = nxt_row;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) cur_v[b] = nxt_v[b];
+      fetch(cb + 1, nxt_row, nxt_v);
     }
   }
 

@@ -18,13 +18,17 @@
 //          depth is a multiple of 8, so slot q % depth always belongs to the same warp, which has
 //          finished item q - depth before it waits for item q: a parity wait can never match a
 //          phase from two fills earlier.
-//   warp 9 (compaction): per chunk, ballots the 16 keep flags, publishes the count, finds the
-//          output offset by decoupled look-back over epoch-tagged status words and scatters idx
-//          and a_val, while the consumers already work on later chunks.
+//          The last consumer warp to finish a chunk publishes the chunk's count (its look-back
+//          aggregate) at once, so other CTAs' look-backs never wait on this CTA's compaction warp.
+//   warp 9 (compaction): per chunk, ballots the 16 keep flags, finds the output offset by a
+//          warp-parallel decoupled look-back over epoch-tagged status words, publishes the
+//          inclusive prefix and scatters idx and a_val, while the consumers work on later chunks.
 //
-// Tickets are taken in increasing order by running CTAs only, and each CTA compacts its chunks
-// in ticket order, so the smallest unfinished chunk can always finish: the look-back never waits
-// on work that cannot progress.  Every wait is bounded (tma.cuh, common.cuh).
+// CTA b's first chunk is chunk b; later chunks come from a ticket counter, in increasing order,
+// to running CTAs only, and each CTA compacts its chunks in order, so the smallest unfinished
+// chunk can always finish: the look-back never waits on work that cannot progress.  The producer
+// starts streaming while the consumers stage the tokens.  Every wait is bounded (tma.cuh,
+// common.cuh).
 #include "common.cuh"
 #include "gemv.cuh"
 #include "kernels.h"
@@ -35,7 +39,7 @@ namespace csffn {
 constexpr int kTmaConsumers = 8;
 constexpr int kTmaThreads = (kTmaConsumers + 2) * kWarp;  // + producer warp + compaction warp
 constexpr int kMaxRingSlots = 32;
-constexpr int kChunkBufs = 4;
+constexpr int kChunkBufs = 8;
 constexpr size_t kTmaSmemBudget = 220 * 1024;
 
 struct GateTmaShared {
@@ -46,6 +50,8 @@ struct GateTmaShared {
   int slot_chunk[kMaxRingSlots];
   int res_chunk[kChunkBufs];
   uint32_t res_keep[kChunkBufs][kChunkRows];
+  uint32_t res_cnt[kChunkBufs];     // kept rows of the chunk so far
+  uint32_t res_arrived[kChunkBufs]; // consumer slots of the chunk finished so far
   int abort;
   uint32_t epoch;
 };
@@ -68,7 +74,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
   XT* xs = reinterpret_cast<XT*>(smem_raw);
   unsigned char* ring = smem_raw + x_bytes;
 
-  stage_tokens<XT, NB>(xs, reinterpret_cast<const XT*>(p.x), p.B, K);
   if (tid == 0) {
     for (int i = 0; i < nslots; ++i) {
       mbar_init(&sh.full[i], 1);
@@ -77,6 +82,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
     for (int i = 0; i < kChunkBufs; ++i) {
       mbar_init(&sh.chunk_full[i], kSlotsPerChunk);
       mbar_init(&sh.chunk_empty[i], 1);
+      sh.res_cnt[i] = 0u;
+      sh.res_arrived[i] = 0u;
     }
     sh.abort = 0;
     sh.epoch = *reinterpret_cast<volatile uint32_t*>(&p.ctl->epoch);
@@ -98,13 +105,13 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
     if (lane == 0) {
       const WT* W = reinterpret_cast<const WT*>(p.W);
       int q = 0;
-      int c_next = (int)atomicAdd(&p.ctl->ticket, 1u);
+      int c_next = (int)blockIdx.x;  // first chunk: no ticket needed
       bool ok = true;
       for (bool done = false; !done && ok;) {
         const int c = c_next;
         done = c >= n_chunks;
         if (c == 0 && n_chunks == 0) *p.count = 0;  // empty row set
-        if (!done) c_next = (int)atomicAdd(&p.ctl->ticket, 1u);
+        if (!done) c_next = (int)gridDim.x + (int)atomicAdd(&p.ctl->ticket, 1u);
         for (int g = 0; g < kSlotsPerChunk; ++g, ++q) {
           const int slot = q % nslots;
           if (!(ok = mbar_wait(&sh.empty[slot], ((q / nslots) & 1) ^ 1, p.err, abort))) break;
@@ -140,14 +147,22 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
     // ------------------------------------------------------------------ consumers
     constexpr int R = kRowsPerSlot;
     const int NV = K / EPV;
+    {  // stage the tokens (consumer warps only; the producer is already streaming)
+      const int per_tok = (int)((size_t)K * sizeof(XT) / 16);
+      uint4* dst = reinterpret_cast<uint4*>(xs);
+      const uint4* src = reinterpret_cast<const uint4*>(p.x);
+      for (int e = tid; e < NB * per_tok; e += kTmaConsumers * kWarp)
+        dst[e] = (e / per_tok) < p.B ? src[e] : make_uint4(0u, 0u, 0u, 0u);
+      asm volatile("bar.sync 1, %0;" ::"n"(kTmaConsumers * kWarp) : "memory");
+    }
     for (int q = warp;; q += kTmaConsumers) {
       const int slot = q % nslots;
       if (!mbar_wait(&sh.full[slot], (q / nslots) & 1, p.err, abort)) break;
       const int c = sh.slot_chunk[slot];
       const int s = q / kSlotsPerChunk;  // this CTA's chunk sequence number
       const int cb = s % kChunkBufs;
-      if (!mbar_wait(&sh.chunk_empty[cb], ((s / kChunkBufs) & 1) ^ 1, p.err, abort)) break;
       if (c < 0) {  // sentinel chunk: tell the compaction warp to stop
+        if (!mbar_wait(&sh.chunk_empty[cb], ((s / kChunkBufs) & 1) ^ 1, p.err, abort)) break;
         if (q % kSlotsPerChunk == 0 && lane == 0) sh.res_chunk[cb] = -1;
         __syncwarp();
         if (lane == 0) {
@@ -160,11 +175,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
       const int pos = (q % kSlotsPerChunk) * R;  // first row of this slot within the chunk
       const int j0 = c * kChunkRows + pos;
       const WT* rows = reinterpret_cast<const WT*>(ring + (size_t)slot * slot_bytes);
-      float acc[R][NB];
+      // Two partial sums per (row, token) halve the dependent FMA chain.
+      float acc2[R][NB][2];
 #pragma unroll
       for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc2[r][b][0] = acc2[r][b][1] = 0.f;
 #pragma unroll 4
       for (int v = lane; v < NV; v += kWarp) {
         float wf[R][EPV];
@@ -180,9 +196,18 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
 #pragma unroll
           for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[r][b] = fmaf(wf[r][e], xf[e], acc[r][b]);
+            for (int e = 0; e < EPV; ++e) acc2[r][b][e & 1] = fmaf(wf[r][e], xf[e], acc2[r][b][e & 1]);
         }
       }
+      // The slot's data is in registers: hand the slot back to the producer before anything else.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[slot]);
+      float acc[R][NB];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[r][b] = acc2[r][b][0] + acc2[r][b][1];
+      if (!mbar_wait(&sh.chunk_empty[cb], ((s / kChunkBufs) & 1) ^ 1, p.err, abort)) break;
       warp_reduce_all<R, NB>(acc);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -215,7 +240,16 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
       if (pos == 0 && lane == 0) sh.res_chunk[cb] = c;
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sh.empty[slot]);
+        uint32_t kept = 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) kept += sh.res_keep[cb][pos + r];
+        atomicAdd(&sh.res_cnt[cb], kept);
+        __threadfence_block();  // the count is in before this slot is counted as finished
+        if (atomicAdd(&sh.res_arrived[cb], 1u) == (uint32_t)(kSlotsPerChunk - 1)) {
+          // last slot of the chunk: publish the aggregate now (chunk 0: its inclusive prefix)
+          const uint32_t agg = atomicAdd(&sh.res_cnt[cb], 0u);
+          st_status(&p.status[c], status_word(epoch, c == 0 ? kFlagInclusive : kFlagAggregate, agg));
+        }
         mbar_arrive(&sh.chunk_full[cb]);
       }
     }
@@ -229,7 +263,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
       const bool keep = lane < kChunkRows && sh.res_keep[cb][lane] != 0u;
       const uint32_t mask = __ballot_sync(0xffffffffu, keep);
       const uint32_t agg = __popc(mask);
-      const uint32_t prefix = warp_lookback(p.status, c, epoch, agg, p.err, lane);
+      const uint32_t prefix = warp_lookback(p.status, c, epoch, agg, p.err, lane, /*agg_published=*/true);
       if (keep) {
         const uint32_t pos = prefix + __popc(mask & ((1u << lane) - 1u));
         if (pos < (uint32_t)p.h) {
@@ -243,7 +277,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gate_tma_kernel(const GateArgs
       }
       if (c == n_chunks - 1 && lane == 0) *p.count = (int32_t)(prefix + agg);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.chunk_empty[cb]);
+      if (lane == 0) {
+        sh.res_cnt[cb] = 0u;
+        sh.res_arrived[cb] = 0u;
+        mbar_arrive(&sh.chunk_empty[cb]);
+      }
     }
   }
 

@@ -36,10 +36,14 @@ cudaError_t launch_gate_compact(const GateArgs& a, int wdtype, bool x_f32, int m
 // four 2-row slots beside the staged tokens in shared memory.
 bool gate_tma_supported(int K, int B, int wdtype, bool x_f32);
 cudaError_t launch_gate_tma(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
-// Picks the bulk-copy kernel when the shape allows it, else the register-streaming one.
+// Streaming version with an asynchronous compaction warp (gate_stream.cu); needs the staged tokens
+// to fit in shared memory.
+bool gate_stream_supported(int K, int B, int wdtype, bool x_f32);
+cudaError_t launch_gate_stream(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
+// Picks the streaming kernel when the shape allows it, else the chunk-synchronous one.
 inline cudaError_t launch_gate(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s) {
-  return gate_tma_supported(a.K, a.B, wdtype, x_f32) ? launch_gate_tma(a, wdtype, x_f32, mode, s)
-                                                     : launch_gate_compact(a, wdtype, x_f32, mode, s);
+  return gate_stream_supported(a.K, a.B, wdtype, x_f32) ? launch_gate_stream(a, wdtype, x_f32, mode, s)
+                                                        : launch_gate_compact(a, wdtype, x_f32, mode, s);
 }
 
 // v[b*h + j] = a_val[b*h + j] * (x_b . W_up[idx[j]]) for j < *count.
@@ -98,6 +102,36 @@ struct RowGemvArgs {
   int transpose_out;  // write y[row*y_stride + b] instead
 };
 cudaError_t launch_row_gemv(const RowGemvArgs& a, int wdtype, bool x_f32, cudaStream_t s);
+
+// One-launch CATS decode step (cats_fused.cu): gate + threshold + up, grid barrier, gathered down
+// projection and compaction of idx / a_val / count.
+struct FusedArgs {
+  const void* W_gate;
+  const void* W_up;
+  const void* W_down_t;
+  const void* x;
+  int d, h, B;
+  const float* bias;
+  float t;
+  int act;
+  float* v;          // [B, h] scratch: a * u per neuron
+  float* afull;      // [B, h] scratch: kept activation per neuron
+  uint8_t* flags;    // [h] scratch: keep flag per neuron
+  float* partial;    // [ranges, B, d] scratch
+  uint32_t* slice_ctr;
+  uint32_t* ctl;        // fused control words (tile counter, exit counter)
+  uint32_t* range_cnt;  // [2][kMaxRowRanges]: rows counted, rows kept per neuron range
+  uint32_t* tickets;    // [64 * 32] row-ticket counters, 128 bytes apart
+  uint32_t* err;
+  int32_t* idx;
+  int32_t* count;
+  float* a_val;
+  void* out;
+  int out_mode;
+  int slices, ranges;  // set by the launcher
+};
+bool cats_fused_supported(int d, int B, int wdtype);
+cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
 
 // Radix selection and per-neuron selection (calibration).
 size_t kth_state_bytes();

@@ -143,6 +143,19 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
                                       const int32_t* idx, const int32_t* count, const float* a_val,
                                       void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
 
+/* One CATS decode step in a single kernel launch: everything csffn_gate_mask followed by
+ * csffn_sparse_ffn_forward computes, with the same outputs (idx, *count, a_val as gate_mask;
+ * out as sparse_ffn_forward).  [CATS] abstract: the gate GEMV, the compare and the flag-gated
+ * GEMV of one FFN layer.  The gate, threshold and up projection of each kept row run in one
+ * pass; after a grid-wide barrier (cooperative launch) the down projection reads only the kept
+ * rows, and idx / a_val / count are compacted.  One launch pays one ramp-up and one tail instead
+ * of three.  Runs for 1 <= B <= 4 with B*d*elem <= 48 KB; other shapes fall back to the two-call
+ * path inside this call.  ws sized by csffn_workspace_size for this layer and batch.  B == 0:
+ * writes *count = 0. */
+csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
+                                    int32_t* idx, int32_t* count, float* a_val,
+                                    void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
 /* Dense gated FFN over all h neurons (the full model that verifies a chunk of
  * sparse-drafted tokens, [SIRIUS] "Approach"; also the speed-up baseline).
  *   out = (act(x W_gate^T + beta) * (x W_up^T)) W_down.  B == 0: no-op.

@@ -215,3 +215,86 @@ def test_llama3_70b_dense_verify_chunk():
     spec, x, _ = synth.llama3_70b_swiglu(n_eval=16, n_calib=1)
     out = run_dense(dev_layer(spec), x)
     assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16
+
+
+# ------------------------------------------------------------------------------ one-launch decode step
+
+def run_fused(layer, x_np, t, out_dtype=torch.float32, ws=None):
+    x = dev(x_np if x_np.ndim == 2 else x_np[None, :])
+    B = x.shape[0]
+    idx = torch.full((layer.h,), -1, dtype=torch.int32, device="cuda")
+    count = torch.full((1,), -7, dtype=torch.int32, device="cuda")
+    a_val = torch.zeros(B, layer.h, dtype=torch.float32, device="cuda")
+    out = torch.full((B, layer.d), float("nan"), dtype=out_dtype, device="cuda")
+    ws = ws if ws is not None else cs.new_workspace(layer, B)
+    cs.cats_ffn_forward(layer, x, t, idx, count, a_val, out, ws)
+    assert cs.check_status(ws) == 0
+    n = int(count.item())
+    return (idx[:n].cpu().numpy(), a_val[:, :n].cpu().numpy().astype(np.float64),
+            out.float().cpu().numpy().astype(np.float64))
+
+
+@pytest.mark.parametrize("d,h,B,dtype,s", [(256, 688, 1, "f32", 0.5), (520, 1000, 3, "bf16", 0.5),
+                                           (4096, 11008, 1, "bf16", 0.5), (4096, 11008, 1, "bf16", 0.9),
+                                           (4096, 14336, 4, "bf16", 0.5), (64, 16, 2, "bf16", 0.3),
+                                           (8192, 2048, 1, "bf16", 0.7), (1024, 777, 8, "bf16", 0.5)])
+def test_fused_decode_matches_oracle_and_two_call_path(d, h, B, dtype, s):
+    spec = synth.make_layer(62, d, d, h, dtype)
+    x = synth.make_tokens(62, d, synth.ROLE_EVAL, B, d, dtype, rms_normalise=dtype == "bf16")
+    a_ref = oracle.gate_activation(x, spec)
+    t = float(np.quantile(np.abs(a_ref), s))
+    layer = dev_layer(spec)
+    idx, a_val, out = run_fused(layer, x, t)
+    assert_index_list(idx, h)
+    band = band_rows(a_ref, t)
+    got = np.zeros(h, bool)
+    got[idx] = True
+    assert np.array_equal(got[~band], oracle.union_mask(oracle.cats_mask(a_ref, t))[~band])
+    m = token_masks(idx, a_val, h)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16_F32OUT
+    assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= tol
+    # the two-call path (other kernels, other summation order) gives the same set outside the band,
+    # the same values to rounding, and the same output to rounding
+    idx2, a_val2, bufs = run_gate(layer, x, t)
+    got2 = np.zeros(h, bool)
+    got2[idx2] = True
+    assert np.array_equal(got[~band], got2[~band])
+    if np.array_equal(idx, idx2):
+        np.testing.assert_allclose(a_val, a_val2, rtol=1e-5, atol=1e-7 * np.abs(a_ref).max())
+    out2 = run_sparse(layer, bufs)
+    m2 = token_masks(idx2, a_val2, h)
+    assert oracle.rel_l2(out2, oracle.sparse_ffn(x, spec, m2)) <= tol
+
+
+def test_fused_decode_repeated_and_modes():
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=64)
+    t = oracle.calibrate_global(xc, spec, 0.5)
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 1)
+    first = run_fused(layer, x[:1], t, ws=ws)
+    for _ in range(10):  # the grid barrier and slice counters reset themselves between launches
+        again = run_fused(layer, x[:1], t, ws=ws)
+        assert np.array_equal(first[0], again[0]) and np.array_equal(first[2], again[2])
+    idx, a_val, outb = run_fused(layer, x[:1], t, out_dtype=torch.bfloat16, ws=ws)
+    m = token_masks(idx, a_val, spec.h)
+    assert oracle.rel_l2(outb, oracle.sparse_ffn(x[:1], spec, m)) <= TOL_BF16
+    # accumulate mode adds into the residual
+    res = torch.ones(1, spec.d, dtype=torch.float32, device="cuda")
+    xd = dev(x[:1])
+    bidx = torch.zeros(spec.h, dtype=torch.int32, device="cuda")
+    bcnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bav = torch.zeros(1, spec.h, device="cuda")
+    cs.cats_ffn_forward(layer, xd, t, bidx, bcnt, bav, res, ws, out_mode=cs._abi.OUT_F32_ACCUMULATE)
+    assert cs.check_status(ws) == 0
+    assert oracle.rel_l2(res.double().cpu().numpy() - 1.0, first[2]) <= TOL_BF16_F32OUT
+
+
+def test_fused_decode_empty_and_all_active():
+    spec = synth.make_layer(63, 0, 512, 700, "bf16")
+    x = synth.make_tokens(63, 0, synth.ROLE_EVAL, 1, 512, "bf16", rms_normalise=True)
+    layer = dev_layer(spec)
+    idx, a_val, out = run_fused(layer, x, 1e9)
+    assert len(idx) == 0 and np.all(out == 0.0)
+    idx, a_val, out = run_fused(layer, x, -1.0)
+    assert len(idx) == spec.h
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16_F32OUT
