@@ -240,9 +240,9 @@ class DecodeBuffers:
 
 
 def cats_decode(layer: FFNLayer, x: torch.Tensor, t: float, out: torch.Tensor, buf: DecodeBuffers,
-                out_mode: Optional[int] = None, stream=None, one_launch: bool = False) -> None:
-    """One CATS sparse FFN step: csffn_gate_mask then csffn_sparse_ffn_forward, or with
-    one_launch the single-kernel csffn_cats_ffn_forward (same outputs)."""
+                out_mode: Optional[int] = None, stream=None, one_launch: bool = True) -> None:
+    """One CATS sparse FFN step: the single-launch csffn_cats_ffn_forward, or with
+    one_launch=False csffn_gate_mask then csffn_sparse_ffn_forward (same outputs)."""
     if one_launch:
         cats_ffn_forward(layer, x, t, buf.idx, buf.count, buf.a_val, out, buf.ws, out_mode=out_mode, stream=stream)
         return

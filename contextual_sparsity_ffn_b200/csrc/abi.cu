@@ -234,13 +234,11 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   a.bias = layer->gate_bias;
   a.t = t;
   a.act = layer->act;
-  a.v = at<float>(ws, L.vbuf);
   a.afull = at<float>(ws, L.afull);
   a.flags = at<uint8_t>(ws, L.flags);
   a.partial = at<float>(ws, L.partial);
-  a.slice_ctr = at<uint32_t>(ws, L.slice_ctr);
+  a.partial_rows = partial_rows(B);
   a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
-  a.range_cnt = at<uint32_t>(ws, L.range_cnt);
   a.tickets = at<uint32_t>(ws, L.tickets);
   a.err = at<uint32_t>(ws, L.err);
   a.idx = idx;

@@ -1,74 +1,69 @@
-// One-launch CATS decode step: gate + threshold + up (phase A), grid barrier, gathered down
-// projection and active-list compaction (phase B).
+// One-launch CATS decode step: gate, threshold, up and down projection in a single pass over the
+// neuron rows, then one cross-CTA sum and the compaction of the active list.
 //
-// "CATS: Contextually-Aware Thresholding for Sparsity in Large Language Models", abstract: the
-// gate GEMV, the compare and the flag-gated GEMV of its custom kernel; here all of one decode step
-// of an FFN layer runs in a single persistent grid.  A decode step reads a few hundred MB, and a
-// separate launch per stage pays its ramp-up and tail every time (measured on B200: a bare
-// 45 MB row stream reaches 3.6 TB/s, a 720 MB one 6.8 TB/s), so the stages share one launch.
+// "CATS: Contextually-Aware Thresholding for Sparsity in Large Language Models", abstract and the
+// section on the custom kernel: the gate GEMV, the compare against t and the flag-gated up and
+// down GEMVs.  Here every stage of one decode step of an FFN layer runs in one persistent grid.
+// A decode step reads a few hundred MB, and a separate launch per stage pays its ramp-up and tail
+// each time (measured on B200: a bare 45 MB row stream reaches 3.6 TB/s, a 720 MB one 6.8 TB/s),
+// and a statically partitioned stream ends in a long tail (CTAs with equal shares finished up to
+// 2.5x apart), so the rows are handed out dynamically in small chunks.
 //
-// Phase A: warp per neuron row; rows come one at a time from ticket counters (an up row follows
-//   only a kept gate row, so static shares would be uneven).  The warp reduces W_gate[r] against
-//   the tokens staged in shared memory, applies bias, activation and the threshold per token,
-//   writes the keep flag and the kept activations, and if any token keeps the row streams W_up[r]
-//   at once and writes v[b, r] = a[b, r] * u[b, r].  It then counts the row (and whether it was
-//   kept) for its neuron range with a release increment.
-// Phase B (dataflow, no grid barrier): a CTA whose warps find no more rows takes phase-B tiles in
-//   range order from a tile counter.  Tile (range q, slice s) waits (bounded) until every row of
-//   range q has been counted, then its warps ballot the range's flags word by word and stream the
-//   slice (16 bytes per lane) of each kept row of W_down^T, accumulating v[b, r] * W_down^T[r, s]
-//   in registers; warps reduce in shared memory, the tile writes one partial per (range, token,
-//   column), and the last tile of a slice sums the partials in range order (deterministic).  The
-//   slice-0 tile of a range also writes the range's part of idx / a_val at the offset given by the
-//   kept counts of the earlier ranges (once those are complete), and the last range writes count.
-//   Ranges complete roughly in order (tickets hand out rows in increasing order), so phase B of
-//   the early ranges runs while phase A finishes the late rows.
-// Every row is owned by a running warp before any CTA waits on a range, so nothing here depends on
-// CTAs that have not started; all waits are bounded.  The last CTA to finish resets the counters.
+// Chunks of kChunk neuron rows come from ticket counters (one per contiguous block of chunks).
+// The chunk's W_gate rows (contiguous) arrive in shared memory by one bulk copy issued while the
+// previous chunk is still being worked on, so every CTA keeps a chunk of gate rows in flight beside
+// its register loads.  For its chunk a CTA
+//   1. has warp w reduce gate row r = chunk row w against the tokens (both in shared memory), add
+//      the bias, apply the activation and the threshold per token, and record the keep flag and
+//      the kept activations; then (block barrier, gate buffer free) thread 0 issues the next
+//      chunk's bulk copy;
+//   2. has the warp of a kept row stream W_up[r] from HBM and form v[b] = a[b] * u[b];
+//   3. (block barrier) streams the kept rows of W_down^T: warp w owns a fixed 1/8 of the d output
+//      columns and accumulates v[b] * W_down^T[r, its columns] in registers over all its chunks,
+//      so no atomics and no cross-warp traffic are needed until the end.
+// When the tickets run out each CTA writes its register partial of out (fp32 [B, d]).  After a
+// grid-wide count (all CTAs are co-resident: cooperative launch) half of each CTA's warps sum the
+// partials in 16-column slices while the other half compact the active list from the keep flags:
+// CTA k takes a fixed range of 32-row words, counts the flags before it, and writes idx / a_val in
+// ascending neuron order.  Every wait is bounded; the last CTA out resets the counters.
 #include "common.cuh"
 #include "gemv.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace csffn {
 
 constexpr int kFusedThreads = 256;
 constexpr int kFusedWarps = kFusedThreads / kWarp;
-constexpr int kFusedWordBlock = 256;  // 32-neuron words compacted per pass in phase B
-// Row tickets: counter i hands out rows i, i + kTicketCounters, ... to the warps with
-// gw % kTicketCounters == i; the counters sit kTicketStride words (128 bytes) apart so that the
-// warps' atomics spread over L2 instead of serialising on one address.
-constexpr int kTicketCounters = 64;
-constexpr int kTicketStride = 32;
+constexpr int kChunk = kFusedWarps;  // neuron rows per chunk, one per warp
+constexpr int kCounters = 32;        // ticket counters
+constexpr int kCounterStride = 32;   // 32-bit words between counters (128 bytes)
+constexpr int kSumCols = 16;         // columns per slice of the final cross-CTA sum
 
-__device__ __forceinline__ uint8_t ld_cg_u8(const uint8_t* p) { return __ldcg(p); }
-
+// Fused control words (FusedArgs::ctl).
+constexpr int kCtlDone = 0;  // CTAs whose partials and flags are written
+constexpr int kCtlExit = 1;  // CTAs finished
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 
-// Bounded wait until *p >= target (acquire).  Returns false after a second (error recorded).
-__device__ __forceinline__ bool wait_at_least(const uint32_t* p, uint32_t target, uint32_t* err) {
-  if (ld_acquire_u32(p) >= target) return true;
+// Bounded wait until *p >= target (acquire).  Gives up after a second and records the timeout.
+__device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* err) {
+  if (ld_acquire_u32(p) >= target) return;
   const uint64_t t0 = globaltimer_now();
   while (ld_acquire_u32(p) < target) {
     if (globaltimer_now() - t0 > 1000000000ull) {
       atomicOr(err, kDevErrTimeout);
-      return false;
+      return;
     }
     __nanosleep(64);
   }
-  return true;
 }
 
-// Dot products of one row with the staged tokens: acc[b] += W[row] . x_b (this lane's share).
+// acc[b] += W[row] . x_b over this lane's share (U 16-byte vectors in flight per lane).
 template <typename WT, int NB, int U>
 __device__ __forceinline__ void row_dot(const WT* __restrict__ row, const WT* __restrict__ xs, int K, int lane,
                                         float (&acc)[NB]) {
@@ -99,303 +94,406 @@ __device__ __forceinline__ void row_dot(const WT* __restrict__ row, const WT* __
   }
 }
 
-// Rows of one 32-neuron word consumed per phase-B batch (two batches in flight per warp).
-template <int NB> struct FusedDownU { static constexpr int value = NB <= 2 ? 4 : 2; };
+template <int NB> struct FusedGateU { static constexpr int value = NB <= 2 ? 16 : 8; };
+// Kept rows whose W_down^T slices are loaded together.
+template <int KD> struct FusedDownRows { static constexpr int value = KD <= 2 ? 4 : 2; };
 
-// Range (of p.ranges) holding 32-neuron word w when n_words words are split evenly.
-__device__ __forceinline__ int range_of_word(int w, int n_words, int ranges) {
-  return (int)(((long long)(w + 1) * ranges - 1) / n_words);
+// Tickets, drawn by thread 0.  Counter g hands out the chunks of block g, [lo(g), lo(g + 1)); a
+// counter found dry is flagged (word 1 of its line) and the thread moves on to the next counter
+// not flagged.  resolve() returns -1 once every counter is dry.
+struct Tickets {
+  uint32_t* ctr;
+  int n_chunks, G;
+  __device__ int lo(int g) const { return (int)((long long)n_chunks * g / G); }
+  __device__ uint32_t draw(int g) const { return atomicAdd(ctr + g * kCounterStride, 1u); }
+  __device__ int resolve(int& g, uint32_t t) const {
+    for (;;) {
+      const int c = lo(g) + (int)t;
+      if (c < lo(g + 1)) return c;
+      ctr[g * kCounterStride + 1] = 1u;
+      uint32_t live = 0;  // bit i: counter i not flagged dry
+#pragma unroll
+      for (int i = 0; i < kCounters; ++i)
+        live |= (i < G && i != g && __ldcg(ctr + i * kCounterStride + 1) == 0u) ? 1u << i : 0u;
+      if (!live) return -1;
+      // first live counter after g, cyclically
+      const uint32_t above = g + 1 < kCounters ? live & (~0u << (g + 1)) : 0u;
+      g = __ffs(above ? above : live) - 1;
+      t = draw(g);
+    }
+  }
+};
+
+// acc[b] += W[row] . x_b over this lane's share, row and tokens both in shared memory.
+template <typename WT, int NB>
+__device__ __forceinline__ void smem_row_dot(const WT* row, const WT* xs, int K, int lane, float (&acc)[NB]) {
+  constexpr int EPV = Vec<WT>::N;
+  const int NV = K / EPV;
+#pragma unroll 4
+  for (int v = lane; v < NV; v += kWarp) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)v * EPV);
+    float wf[EPV];
+    unpack(w, wf);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float xf[EPV];
+      load_x<EPV>(xs + (size_t)b * K + (size_t)v * EPV, xf);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) acc[b] = fmaf(wf[e], xf[e], acc[b]);
+    }
+  }
 }
 
-// Fused control words (FusedArgs::ctl, 32-bit each): row-ticket counters sit elsewhere.
-constexpr int kCtlTile = 0;     // phase-B tile counter
-constexpr int kCtlExit = 1;     // CTAs finished
-constexpr int kCtlWords = 2;
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
-template <typename WT, int NB>
-__global__ void __launch_bounds__(kFusedThreads, 4) cats_fused_kernel(const FusedArgs p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+constexpr int kHalf = kFusedThreads / 2;            // threads of each end-phase group
+constexpr int kSumRowsPar = kHalf / (kSumCols / 4);  // partials summed side by side
+constexpr int kSumLoads = (kFusedMaxCtas + kSumRowsPar - 1) / kSumRowsPar;
+
+template <typename WT, int NB, int KD>
+__global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const FusedArgs p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr int EPV = Vec<WT>::N;
-  constexpr int SW = kWarp * EPV;  // columns per phase-B slice
-  constexpr int U = GemvUnroll<NB>::value;
-  constexpr int UD = FusedDownU<NB>::value;
-  __shared__ float red[kFusedWarps][SW];
-  __shared__ uint32_t s_wcnt[kFusedWordBlock];
-  __shared__ uint32_t s_offset;
-  __shared__ int s_tile;
-  __shared__ bool s_last;
+  constexpr int U = FusedGateU<NB>::value;
+  constexpr int DR = FusedDownRows<KD>::value;
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ int s_abort;
+  __shared__ float s_v[2][kChunk][NB];
+  __shared__ uint8_t s_keep[2][kChunk];
+  __shared__ int s_next[2];
+  __shared__ uint32_t s_cnt[kFusedWarps];
+  __shared__ float4 s_sum[kHalf / kWarp][4];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int d = p.d, h = p.h;
-  const int n_words = (h + kWarp - 1) / kWarp;
+  const int d = p.d, h = p.h, B = p.B;
+  const int cpw = d / EPV / kFusedWarps;  // 16-byte columns of W_down^T owned by each warp
   WT* xs = reinterpret_cast<WT*>(smem_raw);
+  WT* gbuf = xs + (size_t)NB * d;  // W_gate rows of the current chunk [kChunk][d]
   const WT* Wg = reinterpret_cast<const WT*>(p.W_gate);
   const WT* Wu = reinterpret_cast<const WT*>(p.W_up);
   const WT* Wd = reinterpret_cast<const WT*>(p.W_down_t);
-  uint32_t* range_done = p.range_cnt;                  // rows counted per range
-  uint32_t* range_kept = p.range_cnt + kMaxRowRanges;  // kept rows per range
+  const uint32_t row_bytes = (uint32_t)(d * sizeof(WT));
 
-  // ---------------------------------------------------------------- phase A: gate + up
-  stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), p.B, d);
-  __syncthreads();
-  // Rows come one at a time from ticket counters, so the data-dependent up rows balance out; the
-  // next ticket is fetched while the current row streams.
-  // A warp whose counter runs dry marks it exhausted (word 1 of the counter's line) and moves to a
-  // counter that still has rows; it leaves phase A only when all counters are dry, so by then every
-  // row belongs to a running warp.
-  const int gw = blockIdx.x * kFusedWarps + warp;
-  int tc = gw % kTicketCounters;
-  auto take = [&](int c) -> int {  // lane 0: next row of counter c (>= h when it is dry)
-    return c + kTicketCounters * (int)atomicAdd(p.tickets + c * kTicketStride, 1u);
+  Tickets tk;
+  tk.ctr = p.tickets;
+  tk.n_chunks = (h + kChunk - 1) / kChunk;
+  tk.G = tk.n_chunks < kCounters ? tk.n_chunks : kCounters;
+  int g = blockIdx.x % tk.G;
+  uint32_t t_pending = 0;  // thread 0: ticket drawn for the chunk after the one in flight
+  auto issue_gate = [&](int c) {  // thread 0: the chunk's W_gate rows -> gbuf, one bulk copy
+    const int r0 = c * kChunk;
+    const uint32_t bytes = (uint32_t)min(kChunk, h - r0) * row_bytes;
+    mbar_arrive_expect_tx(&s_bar, bytes);
+    bulk_load(gbuf, Wg + (size_t)r0 * d, bytes, &s_bar);
   };
-  int r_next = 0;
-  if (lane == 0) r_next = take(tc);
-  r_next = __shfl_sync(0xffffffffu, r_next, 0);
-  for (;;) {
-    if (r_next >= h) {
-      if (lane == 0) p.tickets[tc * kTicketStride + 1] = 1u;
-      const bool dry_lo = __ldcg(p.tickets + lane * kTicketStride + 1) != 0u;
-      const bool dry_hi = __ldcg(p.tickets + (lane + kWarp) * kTicketStride + 1) != 0u;
-      const uint32_t live_lo = __ballot_sync(0xffffffffu, !dry_lo), live_hi = __ballot_sync(0xffffffffu, !dry_hi);
-      if (!live_lo && !live_hi) break;
-      tc = live_lo ? __ffs(live_lo) - 1 : kWarp + __ffs(live_hi) - 1;
-      if (lane == 0) r_next = take(tc);
-      r_next = __shfl_sync(0xffffffffu, r_next, 0);
-      continue;
+
+  if (tid == 0) {
+    s_abort = 0;
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    const int c0 = tk.resolve(g, tk.draw(g));
+    s_next[0] = c0;
+    if (c0 >= 0) {
+      issue_gate(c0);
+      t_pending = tk.draw(g);
     }
-    const int r = r_next;
-    if (lane == 0) r_next = take(tc);
-    float acc[NB];
+  }
+  stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), B, d);
+  __syncthreads();
+
+  float acc[NB][KD][EPV];
 #pragma unroll
-    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-    row_dot<WT, NB, U>(Wg + (size_t)r * d, xs, d, lane, acc);
-    const float beta = p.bias ? p.bias[r] : 0.f;
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int k = 0; k < KD; ++k)
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) acc[b][k][e] = 0.f;
+
+  int chunk = s_next[0];
+  for (int it = 0; chunk >= 0; ++it) {
+    const int buf = it & 1;
+
+    // 1. gate and threshold for row r (one per warp) from the prefetched rows
+    mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
+    const int r = chunk * kChunk + warp;
     float a[NB];
     bool any = false;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const float z = warp_sum(acc[b]) + beta;
-      const float ab = gate_act(z, p.act);
-      const bool kb = b < p.B && fabsf(ab) > p.t;
-      a[b] = kb ? ab : 0.f;
-      any |= kb;
-    }
-    if (lane == 0) {
-      p.flags[r] = any ? 1 : 0;
+    for (int b = 0; b < NB; ++b) a[b] = 0.f;
+    if (r < h) {
+      float z[NB];
 #pragma unroll
-      for (int b = 0; b < NB; ++b)
-        if (b < p.B) p.afull[(size_t)b * h + r] = a[b];
-    }
-    if (any) {
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-      row_dot<WT, NB, U>(Wu + (size_t)r * d, xs, d, lane, acc);
+      for (int b = 0; b < NB; ++b) z[b] = 0.f;
+      smem_row_dot<WT, NB>(gbuf + (size_t)warp * d, xs, d, lane, z);
+      const float beta = p.bias ? __ldg(p.bias + r) : 0.f;
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        const float u = warp_sum(acc[b]);
-        if (lane == 0 && b < p.B) p.v[(size_t)b * h + r] = a[b] * u;
+        const float ab = gate_act(warp_sum(z[b]) + beta, p.act);
+        const bool kb = b < B && fabsf(ab) > p.t;
+        a[b] = kb ? ab : 0.f;
+        any |= kb;
+      }
+      if (lane == 0) {
+        p.flags[r] = any ? 1 : 0;
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          if (b < B) p.afull[(size_t)b * h + r] = a[b];
       }
     }
-    if (lane == 0) {
-      const int q = range_of_word(r / kWarp, n_words, p.ranges);
-      if (any) atomicAdd(&range_kept[q], 1u);
-      atom_add_release_u32(&range_done[q], 1u);  // the row's outputs are visible before it counts
+    __syncthreads();  // gbuf is free: prefetch the next chunk's gate rows
+    if (tid == 0) {
+      const int cn = tk.resolve(g, t_pending);
+      s_next[buf ^ 1] = cn;
+      if (cn >= 0) {
+        fence_proxy_async_smem();
+        issue_gate(cn);
+        t_pending = tk.draw(g);
+      }
     }
-    r_next = __shfl_sync(0xffffffffu, r_next, 0);
+
+    // 2. up for a kept row, straight from HBM
+    float v[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) v[b] = 0.f;
+    if (any) {
+      float u[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) u[b] = 0.f;
+      row_dot<WT, NB, U>(Wu + (size_t)r * d, xs, d, lane, u);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) v[b] = a[b] * warp_sum(u[b]);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) s_v[buf][warp][b] = v[b];
+      s_keep[buf][warp] = any ? 1 : 0;
+    }
+    __syncthreads();
+
+    // 3. kept rows of W_down^T, this warp's columns
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) m |= s_keep[buf][j] ? 1u << j : 0u;
+    const int next = s_next[buf ^ 1];
+    const int row0 = chunk * kChunk;
+    while (m) {
+      int js[DR];
+      uint4 w[DR][KD];
+#pragma unroll
+      for (int q = 0; q < DR; ++q) {
+        js[q] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1u;
+        const WT* row = Wd + (size_t)(row0 + (js[q] < 0 ? 0 : js[q])) * d;
+#pragma unroll
+        for (int k = 0; k < KD; ++k) {
+          const int c = lane + k * kWarp;
+          w[q][k] = (js[q] >= 0 && c < cpw) ? ld_stream(row + (size_t)(warp * cpw + c) * EPV)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < DR; ++q) {
+        if (js[q] < 0) continue;
+#pragma unroll
+        for (int k = 0; k < KD; ++k) {
+          float wf[EPV];
+          unpack(w[q][k], wf);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float vb = s_v[buf][js[q]][b];
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) acc[b][k][e] = fmaf(vb, wf[e], acc[b][k][e]);
+          }
+        }
+      }
+    }
+    chunk = next;
+  }
+
+  // ---------------------------------------------------------------- partials, then a grid count
+  {
+    float* part = p.partial + (size_t)blockIdx.x * B * d;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b < B) {
+#pragma unroll
+        for (int k = 0; k < KD; ++k) {
+          const int c = lane + k * kWarp;
+          if (c < cpw) {
+            float4* dst = reinterpret_cast<float4*>(part + (size_t)b * d + (size_t)(warp * cpw + c) * EPV);
+#pragma unroll
+            for (int e = 0; e < EPV; e += 4)
+              __stcg(dst + e / 4, make_float4(acc[b][k][e], acc[b][k][e + 1], acc[b][k][e + 2], acc[b][k][e + 3]));
+          }
+        }
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    atomicAdd(&p.ctl[kCtlDone], 1u);
+    wait_at_least(&p.ctl[kCtlDone], gridDim.x, p.err);
   }
   __syncthreads();
 
-  // ---------------------------------------------------------------- phase B: down + compaction
-  const int n_tiles = p.slices * p.ranges;
-  for (;;) {
-    if (tid == 0) s_tile = (int)atomicAdd(&p.ctl[kCtlTile], 1u);
-    __syncthreads();
-    const int tile = s_tile;
-    __syncthreads();
-    if (tile >= n_tiles) break;
-    const int q = tile / p.slices, slice = tile % p.slices;  // range-major: early ranges first
-    const int w0 = (int)((long long)n_words * q / p.ranges), w1 = (int)((long long)n_words * (q + 1) / p.ranges);
-    const int rows_q = min(h, w1 * kWarp) - w0 * kWarp;
-    if (tid == 0) wait_at_least(&range_done[q], (uint32_t)rows_q, p.err);
-    __syncthreads();
-    const int c0 = slice * SW + lane * EPV;
-    const bool col_ok = c0 < d;
-    float acc[NB][EPV];
+  if (warp < kHalf / kWarp) {
+    // ------------------------------------------------------------ cross-CTA sum of the partials
+    // Slice s = columns [16 s, 16 s + 16).  Thread (grp, q) adds float4 q of the partials of CTAs
+    // grp, grp + 32, ... (all loads issued together); the 8 groups of a warp are folded with
+    // shuffles, the 4 warps in shared memory.
+    const int q = tid & 3, grp = tid >> 2;
+    const int n_slices = d / kSumCols;
+    for (int s = blockIdx.x; s < n_slices; s += gridDim.x) {
+      for (int b = 0; b < B; ++b) {
+        float4 x4[kSumLoads];
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
+        for (int i = 0; i < kSumLoads; ++i) {
+          const int c = grp + i * kSumRowsPar;
+          x4[i] = c < (int)gridDim.x
+                      ? __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)c * B + b) * d + (size_t)s * kSumCols) + q)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float4 sum = x4[0];
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) acc[b][e] = 0.f;
-
-    // Words w0 + warp, w0 + warp + 8, ...: ballot the word's flags, then stream its kept rows in
-    // batches of UD, two batches in flight; the next word's flags and v are fetched ahead.
-    auto fetch_word = [&](int w, uint32_t& m, float (&vv)[NB]) {
-      const int r = w * kWarp + lane;
-      const bool f = w < w1 && r < h && ld_cg_u8(p.flags + r) != 0;
-      m = __ballot_sync(0xffffffffu, f);
+        for (int i = 1; i < kSumLoads; ++i) {
+          sum.x += x4[i].x;
+          sum.y += x4[i].y;
+          sum.z += x4[i].z;
+          sum.w += x4[i].w;
+        }
 #pragma unroll
-      for (int b = 0; b < NB; ++b) vv[b] = (f && b < p.B) ? __ldcg(p.v + (size_t)b * h + r) : 0.f;
-    };
-    auto fill = [&](int w, uint32_t& mm, uint4 (&wv)[UD], int (&src)[UD]) {
+        for (int o = 4; o < kWarp; o <<= 1) {
+          sum.x += __shfl_xor_sync(0xffffffffu, sum.x, o);
+          sum.y += __shfl_xor_sync(0xffffffffu, sum.y, o);
+          sum.z += __shfl_xor_sync(0xffffffffu, sum.z, o);
+          sum.w += __shfl_xor_sync(0xffffffffu, sum.w, o);
+        }
+        if (lane < 4) s_sum[warp][lane] = sum;
+        named_sync(1, kHalf);
+        if (tid < 4) {
+          float4 t4 = s_sum[0][tid];
 #pragma unroll
-      for (int u = 0; u < UD; ++u) {
-        src[u] = mm ? __ffs(mm) - 1 : -1;
-        mm &= mm - 1u;
-        const int row = w * kWarp + (src[u] < 0 ? 0 : src[u]);
-        wv[u] = (src[u] >= 0 && col_ok) ? ld_stream(Wd + (size_t)row * d + c0) : make_uint4(0u, 0u, 0u, 0u);
-      }
-    };
-    auto consume = [&](const uint4 (&wv)[UD], const int (&src)[UD], const float (&vv)[NB]) {
-#pragma unroll
-      for (int u = 0; u < UD; ++u) {
-        float wf[EPV];
-        unpack(wv[u], wf);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float vb = __shfl_sync(0xffffffffu, vv[b], src[u] < 0 ? 0 : src[u]);
-          if (src[u] >= 0) {
-#pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[b][e] = fmaf(vb, wf[e], acc[b][e]);
+          for (int w = 1; w < kHalf / kWarp; ++w) {
+            const float4 o4 = s_sum[w][tid];
+            t4.x += o4.x;
+            t4.y += o4.y;
+            t4.z += o4.z;
+            t4.w += o4.w;
           }
-        }
-      }
-    };
-    {
-      uint32_t m_cur, m_nxt;
-      float v_cur[NB], v_nxt[NB];
-      int w = w0 + warp;
-      fetch_word(w, m_cur, v_cur);
-      for (; w < w1; w += kFusedWarps) {
-        fetch_word(w + kFusedWarps, m_nxt, v_nxt);
-        uint32_t mm = m_cur;
-        uint4 wa[UD], wb[UD];
-        int sa[UD], sb[UD];
-        fill(w, mm, wa, sa);
-        while (sa[0] >= 0) {
-          fill(w, mm, wb, sb);
-          consume(wa, sa, v_cur);
-          if (sb[0] < 0) break;
-          fill(w, mm, wa, sa);
-          consume(wb, sb, v_cur);
-        }
-        m_cur = m_nxt;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) v_cur[b] = v_nxt[b];
-      }
-    }
-
-    // cross-warp reduction, one partial row per token
-    const int col = slice * SW + tid;
-    for (int b = 0; b < p.B && b < NB; ++b) {
-#pragma unroll
-      for (int bb = 0; bb < NB; ++bb)
-        if (bb == b)
-#pragma unroll
-          for (int e = 0; e < EPV; ++e) red[warp][lane * EPV + e] = acc[bb][e];
-      __syncthreads();
-      if (tid < SW && col < d) {
-        float sum = 0.f;
-#pragma unroll
-        for (int ww = 0; ww < kFusedWarps; ++ww) sum += red[ww][tid];
-        p.partial[((size_t)q * p.B + b) * d + col] = sum;
-      }
-      __syncthreads();
-    }
-
-    // compacted outputs for this range (slice-0 tile), at the offset of the earlier ranges' kept rows
-    if (slice == 0) {
-      if (tid == 0) {
-        uint32_t before = 0;
-        for (int qq = 0; qq < q; ++qq) {
-          const int a0 = (int)((long long)n_words * qq / p.ranges), a1 = (int)((long long)n_words * (qq + 1) / p.ranges);
-          wait_at_least(&range_done[qq], (uint32_t)(min(h, a1 * kWarp) - a0 * kWarp), p.err);
-          before += ld_acquire_u32(&range_kept[qq]);
-        }
-        s_offset = before;
-      }
-      __syncthreads();
-      uint32_t off = s_offset;
-      for (int wb = w0; wb < w1; wb += kFusedWordBlock) {
-        const int we = min(w1, wb + kFusedWordBlock);
-        for (int w = wb + warp; w < we; w += kFusedWarps) {
-          const int r = w * kWarp + lane;
-          const bool f = r < h && ld_cg_u8(p.flags + r) != 0;
-          const uint32_t m = __ballot_sync(0xffffffffu, f);
-          if (lane == 0) s_wcnt[w - wb] = __popc(m);
-        }
-        __syncthreads();
-        if (tid == 0) {
-          uint32_t run = off;
-          for (int w = wb; w < we; ++w) {
-            const uint32_t c = s_wcnt[w - wb];
-            s_wcnt[w - wb] = run;
-            run += c;
-          }
-          s_offset = run;
-        }
-        __syncthreads();
-        for (int w = wb + warp; w < we; w += kFusedWarps) {
-          const int r = w * kWarp + lane;
-          const bool f = r < h && ld_cg_u8(p.flags + r) != 0;
-          const uint32_t m = __ballot_sync(0xffffffffu, f);
-          if (f) {
-            const uint32_t pos = s_wcnt[w - wb] + __popc(m & ((1u << lane) - 1u));
-            if (pos < (uint32_t)h) {
-              p.idx[pos] = r;
-#pragma unroll
-              for (int b = 0; b < NB; ++b)
-                if (b < p.B) p.a_val[(size_t)b * h + pos] = __ldcg(p.afull + (size_t)b * h + r);
+          const size_t o = (size_t)b * d + (size_t)s * kSumCols + tid * 4;
+          if (p.out_mode == CSFFN_OUT_BF16) {
+            bf16* ob = reinterpret_cast<bf16*>(p.out) + o;
+            ob[0] = __float2bfloat16_rn(t4.x);
+            ob[1] = __float2bfloat16_rn(t4.y);
+            ob[2] = __float2bfloat16_rn(t4.z);
+            ob[3] = __float2bfloat16_rn(t4.w);
+          } else {
+            float4* of = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o);
+            if (p.out_mode == CSFFN_OUT_F32_ACCUMULATE) {
+              const float4 prev = *of;
+              t4.x += prev.x;
+              t4.y += prev.y;
+              t4.z += prev.z;
+              t4.w += prev.w;
             }
+            *of = t4;
           }
         }
-        off = s_offset;
-        __syncthreads();
+        named_sync(1, kHalf);
       }
-      if (q == p.ranges - 1 && tid == 0) *p.count = (int32_t)off;
     }
-
-    // the last tile of this slice sums the partials in range order
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&p.slice_ctr[slice], 1u) == (uint32_t)(p.ranges - 1);
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      if (tid < SW && col < d) {
-        for (int b = 0; b < p.B; ++b) {
-          float sum = 0.f;
-          for (int rr = 0; rr < p.ranges; ++rr) sum += __ldcg(p.partial + ((size_t)rr * p.B + b) * d + col);
-          const size_t o = (size_t)b * d + col;
-          if (p.out_mode == CSFFN_OUT_BF16)
-            reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(sum);
-          else if (p.out_mode == CSFFN_OUT_F32)
-            reinterpret_cast<float*>(p.out)[o] = sum;
-          else
-            reinterpret_cast<float*>(p.out)[o] += sum;
-        }
+  } else {
+    // ------------------------------------------------------------ compaction of the active list
+    // CTA k owns the 32-row words [wa, wb); the kept rows before wa are counted from the flag
+    // bytes (each 0 or 1, so the popcount of a 32-bit word of flags counts its kept rows).
+    const int ct = tid - kHalf, cw = warp - kHalf / kWarp;
+    const int n_words = (h + kWarp - 1) / kWarp;
+    const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
+    const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
+    if (wa < wb || blockIdx.x == gridDim.x - 1) {
+      uint32_t before = 0;
+      const uint4* f4 = reinterpret_cast<const uint4*>(p.flags);
+      for (int i = ct; i < wa * 2; i += kHalf) {
+        const uint4 f = __ldcg(f4 + i);
+        before += __popc(f.x) + __popc(f.y) + __popc(f.z) + __popc(f.w);
       }
-      if (tid == 0) p.slice_ctr[slice] = 0u;
+      before = warp_sum_u32(before);
+      if (lane == 0) s_cnt[cw] = before;
+      named_sync(2, kHalf);
+      uint32_t base = 0;
+#pragma unroll
+      for (int w = 0; w < kHalf / kWarp; ++w) base += s_cnt[w];
+      named_sync(2, kHalf);
+      for (int w0 = wa; w0 < wb; w0 += kHalf / kWarp) {
+        const int w = w0 + cw;
+        const int r = w * kWarp + lane;
+        const bool in = w < wb && r < h;
+        const bool f = in && __ldcg(p.flags + r) != 0;
+        float av[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + r) : 0.f;
+        const uint32_t m = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) s_cnt[cw] = __popc(m);
+        named_sync(2, kHalf);
+        uint32_t off = base, total = base;
+#pragma unroll
+        for (int ww = 0; ww < kHalf / kWarp; ++ww) {
+          off += ww < cw ? s_cnt[ww] : 0u;
+          total += s_cnt[ww];
+        }
+        if (f) {
+          const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
+          p.idx[pos] = r;
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            if (b < B) p.a_val[(size_t)b * h + pos] = av[b];
+        }
+        base = total;
+        named_sync(2, kHalf);
+      }
+      if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
     }
   }
 
-  // the last CTA out resets every counter for the next launch
+  // ---------------------------------------------------------------- the last CTA out resets
+  __syncthreads();
   if (tid == 0) {
     __threadfence();
     if (atomicAdd(&p.ctl[kCtlExit], 1u) == gridDim.x - 1) {
-      for (int i = 0; i < kTicketCounters; ++i) {
-        p.tickets[i * kTicketStride] = 0u;
-        p.tickets[i * kTicketStride + 1] = 0u;
+      for (int i = 0; i < kCounters; ++i) {
+        p.tickets[i * kCounterStride] = 0u;
+        p.tickets[i * kCounterStride + 1] = 0u;
       }
-      for (int i = 0; i < 2 * kMaxRowRanges; ++i) p.range_cnt[i] = 0u;
-      p.ctl[kCtlTile] = 0u;
+      p.ctl[kCtlDone] = 0u;
       p.ctl[kCtlExit] = 0u;
       __threadfence();
     }
   }
 }
 
-template <typename WT, int NB>
+// Dynamic shared memory: the staged tokens and one chunk of W_gate rows.
+static size_t fused_smem_bytes(int d, int nb, size_t es) { return (size_t)(nb + kChunk) * d * es; }
+
+// Down-slice width per lane (16-byte columns) for a shape, 0 when the fused kernel does not take it.
+static int fused_kd(int d, int B, int wdtype) {
+  const int epv = wdtype == CSFFN_F32 ? 4 : 8;
+  if (d % (epv * kFusedWarps) != 0 || d % kSumCols != 0) return 0;
+  const int cpw = d / epv / kFusedWarps;
+  const int kd = cpw <= 32 ? 1 : cpw <= 64 ? 2 : cpw <= 128 ? 4 : 0;
+  // register budget: the down accumulators (tokens x kd x epv floats) beside a streamed row
+  if (kd == 0 || batch_tier(B) * kd * epv > 64 || (epv == 8 && kd == 4 && B > 1)) return 0;
+  return kd;
+}
+
+template <typename WT, int NB, int KD>
 static cudaError_t fused_t(FusedArgs a, cudaStream_t s) {
-  auto kern = cats_fused_kernel<WT, NB>;
-  const size_t smem = (size_t)NB * a.d * sizeof(WT);
+  auto kern = cats_fused_kernel<WT, NB, KD>;
+  const size_t smem = fused_smem_bytes(a.d, NB, sizeof(WT));
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -404,37 +502,55 @@ static cudaError_t fused_t(FusedArgs a, cudaStream_t s) {
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kFusedThreads, smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
-  const int grid = sm_count() * occ;
-  constexpr int SW = kWarp * Vec<WT>::N;
-  a.slices = (a.d + SW - 1) / SW;
-  if (a.slices > grid || a.slices > kMaxSlices) return cudaErrorInvalidConfiguration;
-  const int n_words = (a.h + kWarp - 1) / kWarp;
-  a.ranges = grid / a.slices;
-  if (a.ranges > kMaxRowRanges) a.ranges = kMaxRowRanges;
-  if (a.ranges > n_words) a.ranges = n_words;
-  if (a.ranges < 1) a.ranges = 1;
-  kern<<<grid, kFusedThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  if (occ > 2) occ = 2;
+  int grid = sm_count() * occ;
+  if (grid > a.partial_rows / a.B) grid = a.partial_rows / a.B;
+  if (grid < 1) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 bool cats_fused_supported(int d, int B, int wdtype) {
   const size_t es = wdtype == CSFFN_F32 ? 4 : 2;
-  return B >= 1 && B <= 4 && (size_t)batch_tier(B) * d * es <= 48 * 1024;
+  return B >= 1 && B <= kFusedMaxBatch && fused_smem_bytes(d, batch_tier(B), es) <= 200 * 1024 &&
+         fused_kd(d, B, wdtype) > 0;
+}
+
+template <typename WT, int NB>
+static cudaError_t fused_kd_t(const FusedArgs& a, int kd, cudaStream_t s) {
+  switch (kd) {
+    case 1: return fused_t<WT, NB, 1>(a, s);
+    case 2: return fused_t<WT, NB, 2>(a, s);
+    default:
+      if constexpr (Vec<WT>::N == 8 && NB > 1) return cudaErrorInvalidValue;  // rejected by fused_kd
+      else return fused_t<WT, NB, 4>(a, s);
+  }
 }
 
 cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s) {
+  const int kd = fused_kd(a.d, a.B, wdtype);
+  if (kd == 0) return cudaErrorInvalidValue;
   const int t = batch_tier(a.B);
   if (wdtype == CSFFN_F32) {
     switch (t) {
-      case 1: return fused_t<float, 1>(a, s);
-      case 2: return fused_t<float, 2>(a, s);
-      default: return fused_t<float, 4>(a, s);
+      case 1: return fused_kd_t<float, 1>(a, kd, s);
+      case 2: return fused_kd_t<float, 2>(a, kd, s);
+      default: return fused_kd_t<float, 4>(a, kd, s);
     }
   }
   switch (t) {
-    case 1: return fused_t<bf16, 1>(a, s);
-    case 2: return fused_t<bf16, 2>(a, s);
-    default: return fused_t<bf16, 4>(a, s);
+    case 1: return fused_kd_t<bf16, 1>(a, kd, s);
+    case 2: return fused_kd_t<bf16, 2>(a, kd, s);
+    default: return fused_kd_t<bf16, 4>(a, kd, s);
   }
 }
 

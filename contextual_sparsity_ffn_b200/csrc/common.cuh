@@ -39,20 +39,28 @@ struct WsLayout {
   size_t ctl;        // Control[kNumCtl]
   size_t err;        // uint32 error word (+ pad)
   size_t slice_ctr;  // uint32 [kSliceUsers][kMaxSlices]
-  size_t range_cnt;  // uint32 [2][kMaxRowRanges]       kept rows per neuron range (fused path)
-  size_t tickets;    // uint32 [64][32]                 row-ticket counters, 128 B apart (fused path)
+  size_t tickets;    // uint32 [64][32]                 chunk-ticket counters, 128 B apart (fused path)
   size_t status;     // uint64 [kNumCtl][max_chunks]   look-back status words
   size_t control_end;
   size_t vbuf;       // fp32 [max_batch][h]            v = a * u (sparse) or act(z)*u (dense)
   size_t afull;      // fp32 [max_batch][h]            per-neuron kept activations (fused path)
   size_t flags;      // uint8 [h]                      per-neuron keep flags (fused path)
-  size_t partial;    // fp32 [kMaxRowRanges][max_batch][d]
+  size_t partial;    // fp32 [partial_rows(max_batch)][d]
   size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
   size_t total;
   int max_chunks;
 };
 
 constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
+constexpr int kFusedMaxCtas = 320;  // CTAs of the fused step (2 per SM) with a partial each
+constexpr int kFusedMaxBatch = 4;
+
+// Rows of d floats in the partial region.
+__host__ __device__ inline int partial_rows(int max_batch) {
+  const int ranges = kMaxRowRanges * max_batch;
+  const int fused = kFusedMaxCtas * (max_batch < kFusedMaxBatch ? max_batch : kFusedMaxBatch);
+  return ranges > fused ? ranges : fused;
+}
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -62,7 +70,6 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   L.ctl = o;        o += sizeof(Control) * kNumCtl;
   L.err = o;        o += 64;
   L.slice_ctr = o;  o += sizeof(uint32_t) * kSliceUsers * kMaxSlices;
-  L.range_cnt = o;  o += sizeof(uint32_t) * 2 * kMaxRowRanges;
   o = align_up(o, 128);
   L.tickets = o;    o += sizeof(uint32_t) * 64 * 32;
   o = align_up(o, 256);
@@ -76,7 +83,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   o = align_up(o, 256);
   L.flags = o;      o += align_up((size_t)h, 16);
   o = align_up(o, 256);
-  L.partial = o;    o += sizeof(float) * (size_t)kMaxRowRanges * max_batch * d;
+  // partials: one per row range of the sparse/dense forward, or one per CTA of the fused step
+  L.partial = o;    o += sizeof(float) * (size_t)partial_rows(max_batch) * d;
   o = align_up(o, 256);
   L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);
   o = align_up(o, 256);

@@ -103,8 +103,9 @@ struct RowGemvArgs {
 };
 cudaError_t launch_row_gemv(const RowGemvArgs& a, int wdtype, bool x_f32, cudaStream_t s);
 
-// One-launch CATS decode step (cats_fused.cu): gate + threshold + up, grid barrier, gathered down
-// projection and compaction of idx / a_val / count.
+// One-launch CATS decode step (cats_fused.cu): gate + threshold + up + down in one pass over
+// dynamically assigned row chunks, a grid-wide count, the cross-CTA sum and the compaction of
+// idx / a_val / count.
 struct FusedArgs {
   const void* W_gate;
   const void* W_up;
@@ -114,21 +115,18 @@ struct FusedArgs {
   const float* bias;
   float t;
   int act;
-  float* v;          // [B, h] scratch: a * u per neuron
   float* afull;      // [B, h] scratch: kept activation per neuron
-  uint8_t* flags;    // [h] scratch: keep flag per neuron
-  float* partial;    // [ranges, B, d] scratch
-  uint32_t* slice_ctr;
-  uint32_t* ctl;        // fused control words (tile counter, exit counter)
-  uint32_t* range_cnt;  // [2][kMaxRowRanges]: rows counted, rows kept per neuron range
-  uint32_t* tickets;    // [64 * 32] row-ticket counters, 128 bytes apart
+  uint8_t* flags;    // [h] scratch: keep flag per neuron (16-byte aligned)
+  float* partial;    // [partial_rows / B][B, d] scratch: one fp32 partial of out per CTA
+  int partial_rows;  // capacity of partial in rows of d floats
+  uint32_t* ctl;     // fused control words (done and exit counters), zero between launches
+  uint32_t* tickets; // [32 * 32] chunk-ticket counters and dry flags, 128 bytes apart
   uint32_t* err;
   int32_t* idx;
   int32_t* count;
   float* a_val;
   void* out;
   int out_mode;
-  int slices, ranges;  // set by the launcher
 };
 bool cats_fused_supported(int d, int B, int wdtype);
 cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
