@@ -264,6 +264,34 @@ csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, in
   if ((st = check_ws(ws, ws_bytes, L.ybuf)) != CSFFN_OK) return st;
   cudaStream_t s = as_stream(stream);
 
+  if (dense_mma_supported(layer->d, layer->h, B, layer->wdtype)) {  // tensor cores, one pass
+    DenseGateUpArgs g{};
+    g.W_gate = layer->w_gate;
+    g.W_up = layer->w_up;
+    g.x = x;
+    g.d = layer->d;
+    g.h = layer->h;
+    g.B = B;
+    g.bias = layer->gate_bias;
+    g.act = layer->act;
+    g.v = at<float>(ws, L.vbuf);
+    cudaError_t e = launch_dense_gate_up_mma(g, s);
+    if (e != cudaSuccess) return CSFFN_ERR_CUDA;
+    DownArgs dn{};
+    dn.W_down_t = layer->w_down_t;
+    dn.d = layer->d;
+    dn.h = layer->h;
+    dn.B = B;
+    dn.n_host = layer->h;
+    dn.v = g.v;
+    dn.partial = at<float>(ws, L.partial);
+    dn.slice_ctr = at<uint32_t>(ws, L.slice_ctr) + kMaxSlices;
+    dn.out = out;
+    dn.out_mode = out_mode;
+    dn.err = at<uint32_t>(ws, L.err);
+    return cuda_status(launch_down_mma(dn, partial_rows(B) / B, s));
+  }
+
   // Token groups small enough to stage in shared memory (the whole batch when it fits).
   int group = B;
   while (group > 1 && (size_t)batch_tier(group) * layer->d * esize(layer->wdtype) > kMaxDynSmem) group = (group + 1) / 2;

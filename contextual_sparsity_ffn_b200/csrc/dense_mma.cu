@@ -1,0 +1,329 @@
+// Dense FFN of a block of up to 16 tokens on the tensor cores (bf16 in, fp32 accumulate).
+//
+// "Sirius: Contextual Sparsity with Correction for Efficient LLMs", section on the correction
+// step: the full model re-reads a chunk of recent tokens in parallel, so the dense FFN runs on a
+// block of tokens (16 here) instead of one.  At B = 16 the FFN does 16 multiply-adds per weight
+// element: fp32 FMA on the CUDA cores would take longer than streaming the weights, the tensor
+// cores keep it bound by HBM.
+//
+// Gate and up (dense_gate_up_mma_kernel): warp tile = 16 neurons x 16 tokens, mma.sync
+// m16n8k16 with the neurons as M and the tokens as N.  The weight rows stream from HBM straight
+// into A fragments: a dot product may take its k terms in any order, so lane (g, q) loads 16-byte
+// vectors of rows g and g + 8 and the B fragments (tokens, staged in shared memory in 512-column
+// chunks) are read with the same permutation of k.  Epilogue: v[b, i] = act(z + beta) * u.
+//
+// Down (down_mma_kernel): out[b, :] = sum_i v[b, i] W_down^T[i, :] with M = tokens, N = output
+// columns and K = neurons.  W_down^T rows are staged in shared memory (cp.async, three-stage ring of
+// padded rows) and
+// read as B fragments by ldmatrix .trans; v is split into bf16 high and low parts (two MMAs), so
+// the product carries about 16 mantissa bits of v.  Column tiles x neuron ranges, partials
+// summed by the last CTA of each column tile (in range order).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csffn {
+
+constexpr int kMmaThreads = 128;
+constexpr int kMmaWarps = kMmaThreads / kWarp;
+constexpr int kXChunk = 512;                 // token columns staged per step
+constexpr int kXRow = kXChunk + 32;          // shared row stride in elements (1088 B: conflict-free)
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// ------------------------------------------------------------------------------------------
+// Gate and up.  NT token tiles of 8 (B <= 8: 1, else 2).
+// ------------------------------------------------------------------------------------------
+template <int NT>
+__global__ void __launch_bounds__(kMmaThreads, 4) dense_gate_up_mma_kernel(const DenseGateUpArgs p) {
+  __shared__ __align__(128) bf16 xs[2][16 * kXRow];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, q = lane & 3;
+  const int d = p.d, h = p.h, B = p.B;
+  const bf16* Wg = reinterpret_cast<const bf16*>(p.W_gate);
+  const bf16* Wu = reinterpret_cast<const bf16*>(p.W_up);
+  const bf16* xg = reinterpret_cast<const bf16*>(p.x);
+  const int n_ctiles = ((h + 15) / 16 + kMmaWarps - 1) / kMmaWarps;
+  const int n_chunks = (d + kXChunk - 1) / kXChunk;
+
+  // tokens B..15 stay zero in both buffers
+  for (int e = tid; e < 2 * 16 * kXRow / 8; e += kMmaThreads)
+    reinterpret_cast<uint4*>(&xs[0][0])[e] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  auto stage = [&](int c, int buf) {
+    const int c0 = c * kXChunk, vecs = min(kXChunk, d - c0) / 8;
+    for (int e = tid; e < B * vecs; e += kMmaThreads) {
+      const int b = e / vecs, v = e - b * vecs;
+      cp_async16(&xs[buf][b * kXRow + v * 8], xg + (size_t)b * d + c0 + v * 8, 0u);
+    }
+    cp_async_commit();
+  };
+
+  for (int ct = blockIdx.x; ct < n_ctiles; ct += gridDim.x) {
+    const int i0 = (ct * kMmaWarps + warp) * 16;
+    const int r_lo = i0 + g, r_hi = i0 + g + 8;
+    const bool ok_lo = r_lo < h, ok_hi = r_hi < h;
+    const bf16* g_lo = Wg + (size_t)(ok_lo ? r_lo : 0) * d;
+    const bf16* g_hi = Wg + (size_t)(ok_hi ? r_hi : 0) * d;
+    const bf16* u_lo = Wu + (size_t)(ok_lo ? r_lo : 0) * d;
+    const bf16* u_hi = Wu + (size_t)(ok_hi ? r_hi : 0) * d;
+    float zg[NT][4], zu[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) zg[t][e] = zu[t][e] = 0.f;
+
+    stage(0, 0);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      if (c + 1 < n_chunks) {
+        stage(c + 1, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const int c0 = c * kXChunk, w = min(kXChunk, d - c0);
+      const bf16* xb = xs[buf];
+#pragma unroll 1
+      for (int ks = 0; ks < w; ks += 128) {
+        // lane (g, q) holds k = k0 + (4 j + q) * 8 + 0..7 of its rows, j = 0..3 (256 B per row per quad)
+        const size_t k0 = (size_t)c0 + ks;
+        uint4 a_glo[4], a_ghi[4], a_ulo[4], a_uhi[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const size_t off = k0 + (size_t)(4 * j + q) * 8;
+          const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+          a_glo[j] = ok_lo ? ld_stream(g_lo + off) : z4;
+          a_ghi[j] = ok_hi ? ld_stream(g_hi + off) : z4;
+          a_ulo[j] = ok_lo ? ld_stream(u_lo + off) : z4;
+          a_uhi[j] = ok_hi ? ld_stream(u_hi + off) : z4;
+        }
+        uint4 xb4[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            xb4[t][j] = *reinterpret_cast<const uint4*>(xb + (g + 8 * t) * kXRow + ks + (4 * j + q) * 8);
+        // sub-step s: words (u, u + 1) of vector j = s / 2, u = 2 (s % 2); the same words of the
+        // token vectors give the matching B fragment
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int j = s >> 1, u = (s & 1) * 2;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const uint32_t b0 = word(xb4[t][j], u), b1 = word(xb4[t][j], u + 1);
+            mma_16816(zg[t], word(a_glo[j], u), word(a_ghi[j], u), word(a_glo[j], u + 1), word(a_ghi[j], u + 1),
+                      b0, b1);
+            mma_16816(zu[t], word(a_ulo[j], u), word(a_uhi[j], u), word(a_ulo[j], u + 1), word(a_uhi[j], u + 1),
+                      b0, b1);
+          }
+        }
+      }
+      __syncthreads();  // this buffer is restaged two chunks later
+    }
+
+    // C fragment: c[0], c[1] = (row g, tokens 2q, 2q + 1); c[2], c[3] = (row g + 8, same tokens)
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int i = half ? r_hi : r_lo;
+      if (i >= h) continue;
+      const float beta = p.bias ? p.bias[i] : 0.f;
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int b = 8 * t + 2 * q + e;
+          if (b < B) p.v[(size_t)b * h + i] = gate_act(zg[t][2 * half + e] + beta, p.act) * zu[t][2 * half + e];
+        }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Down: out[b, :] = sum_i v[b, i] * W_down^T[i, :] for i < h.
+// CTA tile: 64 output columns x a range of neurons; warp w owns columns 16 w .. 16 w + 15 (two
+// n tiles) for all 16 tokens.  W_down^T rows of the tile (128 B each) are staged 128 neurons at a
+// time in a three-block cp.async ring, in rows padded to 144 B so that ldmatrix reads them without
+// bank conflicts.
+// ------------------------------------------------------------------------------------------
+constexpr int kDnCols = 64;
+constexpr int kDnK = 128;                   // neurons per staged block
+constexpr int kDnStages = 3;                // staged blocks (two in flight while one is used)
+constexpr int kDnRow = kDnCols + 8;         // shared row stride in elements (144 B)
+
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* smem_row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
+}
+
+// fp32 pair -> bf16x2 (round to nearest) and the bf16x2 of what that rounding left out
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+  const float ra = a - __low2float(h2), rb = b - __high2float(h2);
+  const __nv_bfloat162 l2 = __floats2bfloat162_rn(ra, rb);
+  hi = *reinterpret_cast<const uint32_t*>(&h2);
+  lo = *reinterpret_cast<const uint32_t*>(&l2);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs p, int ranges) {
+  extern __shared__ __align__(128) unsigned char dn_smem[];
+  bf16 (*ws)[kDnK * kDnRow] = reinterpret_cast<bf16 (*)[kDnK * kDnRow]>(dn_smem);
+  __shared__ bool s_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, q = lane & 3;
+  const int d = p.d, h = p.h, B = p.B;
+  const bf16* Wd = reinterpret_cast<const bf16*>(p.W_down_t);
+  const int col0 = blockIdx.x * kDnCols;
+  const int ry = blockIdx.y;
+  const int n_rows = p.n_host;
+  const int k_lo = (int)((long long)n_rows * ry / ranges), k_hi = (int)((long long)n_rows * (ry + 1) / ranges);
+  const int n_blocks = (k_hi - k_lo + kDnK - 1) / kDnK;
+
+  auto stage = [&](int blk, int buf) {  // rows k_lo + 64 blk .. of columns col0 .. col0 + 63
+    const int r0 = k_lo + blk * kDnK;
+    for (int e = tid; e < kDnK * (kDnCols / 8); e += kMmaThreads) {
+      const int rr = e >> 3, v = e & 7;
+      bf16* dst = &ws[buf][rr * kDnRow + v * 8];
+      if (r0 + rr < k_hi)
+        cp_async16(dst, Wd + (size_t)(r0 + rr) * d + col0 + v * 8, 0u);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+  };
+
+  float acc[2][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+
+#pragma unroll
+  for (int s0 = 0; s0 < kDnStages - 1; ++s0) {
+    if (s0 < n_blocks) stage(s0, s0);
+    else cp_async_commit();  // empty group: every iteration waits on the same group count
+  }
+  for (int blk = 0; blk < n_blocks; ++blk) {
+    const int buf = blk % kDnStages;
+    if (blk + kDnStages - 1 < n_blocks) stage(blk + kDnStages - 1, (blk + kDnStages - 1) % kDnStages);
+    else cp_async_commit();
+    cp_async_wait<kDnStages - 1>();
+    __syncthreads();
+    const int kb0 = k_lo + blk * kDnK;
+#pragma unroll
+    for (int kk = 0; kk < kDnK; kk += 16) {
+      // A fragment (tokens x neurons) from v: rows g and g + 8, neurons kb0 + kk + 2q (+1, +8, +9)
+      const int kn = kb0 + kk + 2 * q;
+      float va[2][4];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int b = g + 8 * hh;
+        const float* vr = p.v + (size_t)b * h;
+        const bool okb = b < B && NT > hh;
+        va[hh][0] = okb && kn < k_hi ? __ldg(vr + kn) : 0.f;
+        va[hh][1] = okb && kn + 1 < k_hi ? __ldg(vr + kn + 1) : 0.f;
+        va[hh][2] = okb && kn + 8 < k_hi ? __ldg(vr + kn + 8) : 0.f;
+        va[hh][3] = okb && kn + 9 < k_hi ? __ldg(vr + kn + 9) : 0.f;
+      }
+      uint32_t ah[4], al[4];
+      split_bf16x2(va[0][0], va[0][1], ah[0], al[0]);  // row g, k 2q..2q+1
+      split_bf16x2(va[1][0], va[1][1], ah[1], al[1]);  // row g+8
+      split_bf16x2(va[0][2], va[0][3], ah[2], al[2]);  // row g, k 2q+8..
+      split_bf16x2(va[1][2], va[1][3], ah[3], al[3]);  // row g+8
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        // B fragment: neurons kk .. kk + 15 (rows of the staged block), columns 16 warp + 8 t ..
+        uint32_t b0, b1;
+        const int lrow = kk + (lane & 15);
+        ldmatrix_x2_trans(b0, b1, &ws[buf][lrow * kDnRow + warp * 16 + t * 8]);
+        mma_16816(acc[t], ah[0], ah[1], ah[2], ah[3], b0, b1);
+        mma_16816(acc[t], al[0], al[1], al[2], al[3], b0, b1);
+      }
+    }
+    __syncthreads();
+  }
+
+  // partial of this neuron range: C rows = tokens g, g + 8; columns 16 warp + 8 t + 2q (+1)
+  float* part = p.partial + (size_t)ry * B * d;
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = g + 8 * (e >> 1);
+      const int col = col0 + warp * 16 + t * 8 + 2 * q + (e & 1);
+      if (b < B && col < d) __stcg(part + (size_t)b * d + col, acc[t][e]);
+    }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&p.slice_ctr[blockIdx.x], 1u) == (uint32_t)(ranges - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = tid; e < B * kDnCols; e += kMmaThreads) {
+    const int b = e / kDnCols, col = col0 + e % kDnCols;
+    if (col >= d) continue;
+    float sum = 0.f;
+    for (int r = 0; r < ranges; ++r) sum += __ldcg(p.partial + ((size_t)r * B + b) * d + col);
+    const size_t o = (size_t)b * d + col;
+    if (p.out_mode == CSFFN_OUT_BF16)
+      reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(sum);
+    else if (p.out_mode == CSFFN_OUT_F32)
+      reinterpret_cast<float*>(p.out)[o] = sum;
+    else
+      reinterpret_cast<float*>(p.out)[o] += sum;
+  }
+  if (tid == 0) p.slice_ctr[blockIdx.x] = 0u;
+}
+
+// ------------------------------------------------------------------------------------------
+// Launchers
+// ------------------------------------------------------------------------------------------
+bool dense_mma_supported(int d, int h, int B, int wdtype) {
+  return wdtype == CSFFN_BF16 && B >= kDenseMmaMinBatch && B <= 16 && d % 128 == 0 && d % kDnCols == 0 &&
+         d / kDnCols <= kMaxSlices && h >= 16;
+}
+
+cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
+  const int n_ctiles = ((a.h + 15) / 16 + kMmaWarps - 1) / kMmaWarps;
+  int occ = 0;
+  cudaError_t e = a.B <= 8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dense_gate_up_mma_kernel<1>, kMmaThreads, 0)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dense_gate_up_mma_kernel<2>, kMmaThreads, 0);
+  if (e != cudaSuccess) return e;
+  int grid = sm_count() * (occ > 0 ? occ : 1);
+  if (grid > n_ctiles) grid = n_ctiles;
+  if (a.B <= 8)
+    dense_gate_up_mma_kernel<1><<<grid, kMmaThreads, 0, s>>>(a);
+  else
+    dense_gate_up_mma_kernel<2><<<grid, kMmaThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_down_mma(const DownArgs& a, int max_ranges, cudaStream_t s) {
+  const int slices = a.d / kDnCols;
+  const size_t smem = sizeof(bf16) * kDnStages * kDnK * kDnRow;
+  cudaError_t e = cudaFuncSetAttribute(down_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, down_mma_kernel<2>, kMmaThreads, smem);
+  if (e != cudaSuccess) return e;
+  int ranges = sm_count() * (occ > 0 ? occ : 1) / slices;  // one wave
+  if (ranges < 1) ranges = 1;
+  if (ranges > max_ranges) ranges = max_ranges;
+  if (ranges > (a.n_host + kDnK - 1) / kDnK) ranges = (a.n_host + kDnK - 1) / kDnK;
+  dim3 grid(slices, ranges);
+  down_mma_kernel<2><<<grid, kMmaThreads, smem, s>>>(a, ranges);
+  return cudaGetLastError();
+}
+
+}  // namespace csffn

@@ -103,6 +103,13 @@ struct RowGemvArgs {
 };
 cudaError_t launch_row_gemv(const RowGemvArgs& a, int wdtype, bool x_f32, cudaStream_t s);
 
+// Dense FFN of up to 16 tokens on the tensor cores (dense_mma.cu): gate/up into v, then the down
+// projection over all h neurons (DownArgs with idx = count = NULL, n_host = h).
+constexpr int kDenseMmaMinBatch = 8;  // from this many tokens on, FMA throughput would bound the dense FFN
+bool dense_mma_supported(int d, int h, int B, int wdtype);
+cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s);
+cudaError_t launch_down_mma(const DownArgs& a, int max_ranges, cudaStream_t s);
+
 // One-launch CATS decode step (cats_fused.cu): gate + threshold + up + down in one pass over
 // dynamically assigned row chunks, a grid-wide count, the cross-CTA sum and the compaction of
 // idx / a_val / count.
@@ -119,6 +126,7 @@ struct FusedArgs {
   uint8_t* flags;    // [h] scratch: keep flag per neuron (16-byte aligned)
   float* partial;    // [partial_rows / B][B, d] scratch: one fp32 partial of out per CTA
   int partial_rows;  // capacity of partial in rows of d floats
+  int chunk_rows;    // neuron rows per chunk (set by the launcher)
   uint32_t* ctl;     // fused control words (done and exit counters), zero between launches
   uint32_t* tickets; // [32 * 32] chunk-ticket counters and dry flags, 128 bytes apart
   uint32_t* err;

@@ -146,12 +146,15 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
 /* One CATS decode step in a single kernel launch: everything csffn_gate_mask followed by
  * csffn_sparse_ffn_forward computes, with the same outputs (idx, *count, a_val as gate_mask;
  * out as sparse_ffn_forward).  [CATS] abstract: the gate GEMV, the compare and the flag-gated
- * GEMV of one FFN layer.  The gate, threshold and up projection of each kept row run in one
- * pass; after a grid-wide barrier (cooperative launch) the down projection reads only the kept
- * rows, and idx / a_val / count are compacted.  One launch pays one ramp-up and one tail instead
- * of three.  Runs for 1 <= B <= 4 with B*d*elem <= 48 KB; other shapes fall back to the two-call
- * path inside this call.  ws sized by csffn_workspace_size for this layer and batch.  B == 0:
- * writes *count = 0. */
+ * GEMV of one FFN layer.  One pass over dynamically assigned chunks of neuron rows runs the gate,
+ * the threshold, and the up and down projections of the kept rows; after a grid-wide count
+ * (cooperative launch) the per-CTA partial outputs are summed and idx / a_val / count compacted.
+ * One launch pays one ramp-up and one tail instead of three.  Runs for 1 <= B <= 4 when
+ * d % 128 == 0 (bf16; d % 64 for fp32) and the tokens fit in shared memory beside the weight
+ * buffers; other shapes fall back to the two-call path inside this call.  The mask and a_val are
+ * bit-for-bit repeatable; out may differ from launch to launch in the last bits (rows reach CTAs
+ * dynamically, so the order of the final fp32 sum varies).  ws sized by csffn_workspace_size for
+ * this layer and batch.  B == 0: writes *count = 0. */
 csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
                                     int32_t* idx, int32_t* count, float* a_val,
                                     void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
@@ -159,8 +162,11 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
 /* Dense gated FFN over all h neurons (the full model that verifies a chunk of
  * sparse-drafted tokens, [SIRIUS] "Approach"; also the speed-up baseline).
  *   out = (act(x W_gate^T + beta) * (x W_up^T)) W_down.  B == 0: no-op.
- *   bf16 layers with B >= 8 run on the tensor cores (the 16-token verify chunk);
- *   their intermediate activations are rounded to bf16 before the down GEMM. */
+ *   bf16 layers with 8 <= B <= 16, d % 128 == 0 and d <= 8192 run on the tensor cores (the
+ *   16-token verify chunk: bf16 MMA with fp32 accumulation, one pass over the weights for all
+ *   tokens); the down projection takes the fp32 activations as a bf16 high part plus a bf16
+ *   low part, so about 16 of their mantissa bits reach the product.  Other calls run on the
+ *   CUDA cores (fp32 FMA). */
 csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,
                                      void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
 

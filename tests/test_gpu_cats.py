@@ -212,9 +212,30 @@ def test_llama3_70b_batch1_sampled():
 
 
 def test_llama3_70b_dense_verify_chunk():
+    # 16 tokens at d = 8192: the tensor-core path (one pass over W_gate / W_up for all tokens)
     spec, x, _ = synth.llama3_70b_swiglu(n_eval=16, n_calib=1)
     out = run_dense(dev_layer(spec), x)
-    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16
+    assert oracle.rel_l2(out, oracle.dense_ffn(x, spec)) <= TOL_BF16_F32OUT
+
+
+@pytest.mark.parametrize("d,h,B,act", [(1024, 2000, 16, "silu"), (640, 1000, 9, "silu"), (1024, 777, 8, "silu"),
+                                       (4096, 1024, 12, "relu"), (128, 16, 16, "silu"), (2048, 3000, 15, "silu")])
+def test_dense_token_block_tensor_cores(d, h, B, act):
+    """Dense FFN for 8..16 tokens (bf16): tensor-core gate/up and down, ragged neuron tiles,
+    partial 512-column chunks, the ReGLU bias; fp32 output to 1e-4, bf16 output to 1e-2."""
+    bias = (-0.5, 0.3) if act == "relu" else None
+    spec = synth.make_layer(64, d, d, h, "bf16", act, bias_mean_std=bias)
+    x = synth.make_tokens(64, d, synth.ROLE_EVAL, B, d, "bf16", rms_normalise=True)
+    layer = dev_layer(spec)
+    ref = oracle.dense_ffn(x, spec)
+    out = run_dense(layer, x)
+    assert oracle.rel_l2(out, ref) <= TOL_BF16_F32OUT
+    outb = run_dense(layer, x, out_dtype=torch.bfloat16)
+    assert oracle.rel_l2(outb, ref) <= TOL_BF16
+    # each token's row equals its own batch-1 dense output (CUDA-core GEMV path)
+    for b in (0, B - 1):
+        one = run_dense(layer, x[b:b + 1])
+        assert oracle.rel_l2(out[b:b + 1], one) <= TOL_BF16_F32OUT
 
 
 # ------------------------------------------------------------------------------ one-launch decode step
