@@ -350,21 +350,22 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     const int n_slices = d / kSumCols;
     for (int s = blockIdx.x; s < n_slices; s += gridDim.x) {
       for (int b = 0; b < B; ++b) {
+        // every load is issued (rows past the grid read row 0 and are weighted 0), then summed
         float4 x4[kSumLoads];
 #pragma unroll
         for (int i = 0; i < kSumLoads; ++i) {
           const int c = grp + i * kSumRowsPar;
-          x4[i] = c < (int)gridDim.x
-                      ? __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)c * B + b) * d + (size_t)s * kSumCols) + q)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+          const int cc = c < (int)gridDim.x ? c : 0;
+          x4[i] = __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)cc * B + b) * d + (size_t)s * kSumCols) + q);
         }
-        float4 sum = x4[0];
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 1; i < kSumLoads; ++i) {
-          sum.x += x4[i].x;
-          sum.y += x4[i].y;
-          sum.z += x4[i].z;
-          sum.w += x4[i].w;
+        for (int i = 0; i < kSumLoads; ++i) {
+          const float wgt = grp + i * kSumRowsPar < (int)gridDim.x ? 1.f : 0.f;
+          sum.x = fmaf(wgt, x4[i].x, sum.x);
+          sum.y = fmaf(wgt, x4[i].y, sum.y);
+          sum.z = fmaf(wgt, x4[i].z, sum.z);
+          sum.w = fmaf(wgt, x4[i].w, sum.w);
         }
 #pragma unroll
         for (int o = 4; o < kWarp; o <<= 1) {

@@ -13,9 +13,9 @@
 // chunks) are read with the same permutation of k.  Epilogue: v[b, i] = act(z + beta) * u.
 //
 // Down (down_mma_kernel): out[b, :] = sum_i v[b, i] W_down^T[i, :] with M = tokens, N = output
-// columns and K = neurons.  W_down^T rows are staged in shared memory (cp.async, three-stage ring of
-// padded rows) and
-// read as B fragments by ldmatrix .trans; v is split into bf16 high and low parts (two MMAs), so
+// columns and K = neurons.  W_down^T rows and the matching slice of v are staged in shared memory
+// (cp.async, four-block ring, padded rows); W_down^T is read as B fragments by ldmatrix .trans and
+// v is split into bf16 high and low parts (two MMAs), so
 // the product carries about 16 mantissa bits of v.  Column tiles x neuron ranges, partials
 // summed by the last CTA of each column tile (in range order).
 #include "common.cuh"
@@ -152,14 +152,17 @@ __global__ void __launch_bounds__(kMmaThreads, 4) dense_gate_up_mma_kernel(const
 // ------------------------------------------------------------------------------------------
 // Down: out[b, :] = sum_i v[b, i] * W_down^T[i, :] for i < h.
 // CTA tile: 64 output columns x a range of neurons; warp w owns columns 16 w .. 16 w + 15 (two
-// n tiles) for all 16 tokens.  W_down^T rows of the tile (128 B each) are staged 128 neurons at a
-// time in a three-block cp.async ring, in rows padded to 144 B so that ldmatrix reads them without
-// bank conflicts.
+// n tiles) for all 16 tokens.  W_down^T rows of the tile (128 B each) and the tokens' v for the same
+// neurons are staged 64 neurons at a time in a four-block cp.async ring, in rows padded so that
+// ldmatrix and the A-fragment reads are free of bank conflicts.
 // ------------------------------------------------------------------------------------------
 constexpr int kDnCols = 64;
-constexpr int kDnK = 128;                   // neurons per staged block
-constexpr int kDnStages = 3;                // staged blocks (two in flight while one is used)
-constexpr int kDnRow = kDnCols + 8;         // shared row stride in elements (144 B)
+constexpr int kDnK = 64;                    // neurons per staged block
+constexpr int kDnStages = 4;                // staged blocks (three in flight while one is used)
+constexpr int kDnRow = kDnCols + 8;         // W_down^T tile row stride in elements (144 B)
+constexpr int kVRow = kDnK + 8;             // v tile row stride in floats (conflict-free 8-byte reads)
+constexpr size_t kDnWBytes = sizeof(bf16) * kDnK * kDnRow;
+constexpr size_t kDnStageBytes = kDnWBytes + sizeof(float) * 16 * kVRow;
 
 __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* smem_row) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
@@ -179,26 +182,44 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
 template <int NT>
 __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs p, int ranges) {
   extern __shared__ __align__(128) unsigned char dn_smem[];
-  bf16 (*ws)[kDnK * kDnRow] = reinterpret_cast<bf16 (*)[kDnK * kDnRow]>(dn_smem);
   __shared__ bool s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, q = lane & 3;
   const int d = p.d, h = p.h, B = p.B;
   const bf16* Wd = reinterpret_cast<const bf16*>(p.W_down_t);
   const int col0 = blockIdx.x * kDnCols;
   const int ry = blockIdx.y;
-  const int n_rows = p.n_host;
-  const int k_lo = (int)((long long)n_rows * ry / ranges), k_hi = (int)((long long)n_rows * (ry + 1) / ranges);
-  const int n_blocks = (k_hi - k_lo + kDnK - 1) / kDnK;
+  // neuron range of this CTA, in whole blocks (block starts stay 16-byte aligned in v)
+  const int n_blk = (p.n_host + kDnK - 1) / kDnK;
+  const int blk_lo = (int)((long long)n_blk * ry / ranges), blk_hi = (int)((long long)n_blk * (ry + 1) / ranges);
+  const int k_lo = blk_lo * kDnK, k_hi = min(p.n_host, blk_hi * kDnK);
+  const int n_blocks = blk_hi - blk_lo;
+  auto w_tile = [&](int buf) { return reinterpret_cast<bf16*>(dn_smem + (size_t)buf * kDnStageBytes); };
+  auto v_tile = [&](int buf) { return reinterpret_cast<float*>(dn_smem + (size_t)buf * kDnStageBytes + kDnWBytes); };
 
-  auto stage = [&](int blk, int buf) {  // rows k_lo + 64 blk .. of columns col0 .. col0 + 63
+  // token rows B..15 of every staged v tile stay zero
+  for (int e = tid; e < kDnStages * 16 * kVRow; e += kMmaThreads) {
+    const int buf = e / (16 * kVRow), rem = e % (16 * kVRow);
+    if (rem / kVRow >= B) v_tile(buf)[rem] = 0.f;
+  }
+  auto stage = [&](int blk, int buf) {  // neurons k_lo + 64 blk ..: W_down^T columns col0 .. col0 + 63, and v
     const int r0 = k_lo + blk * kDnK;
+    bf16* wt = w_tile(buf);
     for (int e = tid; e < kDnK * (kDnCols / 8); e += kMmaThreads) {
       const int rr = e >> 3, v = e & 7;
-      bf16* dst = &ws[buf][rr * kDnRow + v * 8];
+      bf16* dst = wt + rr * kDnRow + v * 8;
       if (r0 + rr < k_hi)
         cp_async16(dst, Wd + (size_t)(r0 + rr) * d + col0 + v * 8, 0u);
       else
         *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    float* vt = v_tile(buf);
+    for (int e = tid; e < B * (kDnK / 4); e += kMmaThreads) {
+      const int b = e / (kDnK / 4), c = e % (kDnK / 4);
+      float* dst = vt + b * kVRow + c * 4;
+      if (r0 + c * 4 < k_hi)  // h % 4 == 0: a 4-neuron group is wholly in range or wholly out
+        cp_async16(dst, p.v + (size_t)b * h + r0 + c * 4, 0u);
+      else
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     cp_async_commit();
   };
@@ -220,33 +241,26 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
     else cp_async_commit();
     cp_async_wait<kDnStages - 1>();
     __syncthreads();
-    const int kb0 = k_lo + blk * kDnK;
+    const bf16* wt = w_tile(buf);
+    const float* vt = v_tile(buf);
 #pragma unroll
     for (int kk = 0; kk < kDnK; kk += 16) {
-      // A fragment (tokens x neurons) from v: rows g and g + 8, neurons kb0 + kk + 2q (+1, +8, +9)
-      const int kn = kb0 + kk + 2 * q;
-      float va[2][4];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int b = g + 8 * hh;
-        const float* vr = p.v + (size_t)b * h;
-        const bool okb = b < B && NT > hh;
-        va[hh][0] = okb && kn < k_hi ? __ldg(vr + kn) : 0.f;
-        va[hh][1] = okb && kn + 1 < k_hi ? __ldg(vr + kn + 1) : 0.f;
-        va[hh][2] = okb && kn + 8 < k_hi ? __ldg(vr + kn + 8) : 0.f;
-        va[hh][3] = okb && kn + 9 < k_hi ? __ldg(vr + kn + 9) : 0.f;
-      }
+      // A fragment (tokens x neurons) from the staged v: rows g and g + 8, neurons kk + 2q (+1, +8, +9)
+      const float2 v00 = *reinterpret_cast<const float2*>(vt + g * kVRow + kk + 2 * q);
+      const float2 v10 = *reinterpret_cast<const float2*>(vt + (g + 8) * kVRow + kk + 2 * q);
+      const float2 v01 = *reinterpret_cast<const float2*>(vt + g * kVRow + kk + 2 * q + 8);
+      const float2 v11 = *reinterpret_cast<const float2*>(vt + (g + 8) * kVRow + kk + 2 * q + 8);
       uint32_t ah[4], al[4];
-      split_bf16x2(va[0][0], va[0][1], ah[0], al[0]);  // row g, k 2q..2q+1
-      split_bf16x2(va[1][0], va[1][1], ah[1], al[1]);  // row g+8
-      split_bf16x2(va[0][2], va[0][3], ah[2], al[2]);  // row g, k 2q+8..
-      split_bf16x2(va[1][2], va[1][3], ah[3], al[3]);  // row g+8
+      split_bf16x2(v00.x, v00.y, ah[0], al[0]);  // row g, k 2q..2q+1
+      split_bf16x2(v10.x, v10.y, ah[1], al[1]);  // row g+8
+      split_bf16x2(v01.x, v01.y, ah[2], al[2]);  // row g, k 2q+8..
+      split_bf16x2(v11.x, v11.y, ah[3], al[3]);  // row g+8
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         // B fragment: neurons kk .. kk + 15 (rows of the staged block), columns 16 warp + 8 t ..
         uint32_t b0, b1;
         const int lrow = kk + (lane & 15);
-        ldmatrix_x2_trans(b0, b1, &ws[buf][lrow * kDnRow + warp * 16 + t * 8]);
+        ldmatrix_x2_trans(b0, b1, wt + lrow * kDnRow + warp * 16 + t * 8);
         mma_16816(acc[t], ah[0], ah[1], ah[2], ah[3], b0, b1);
         mma_16816(acc[t], al[0], al[1], al[2], al[3], b0, b1);
       }
@@ -291,7 +305,7 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
 // ------------------------------------------------------------------------------------------
 bool dense_mma_supported(int d, int h, int B, int wdtype) {
   return wdtype == CSFFN_BF16 && B >= kDenseMmaMinBatch && B <= 16 && d % 128 == 0 && d % kDnCols == 0 &&
-         d / kDnCols <= kMaxSlices && h >= 16;
+         d / kDnCols <= kMaxSlices && h >= 16 && h % 4 == 0;
 }
 
 cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
@@ -311,7 +325,7 @@ cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
 
 cudaError_t launch_down_mma(const DownArgs& a, int max_ranges, cudaStream_t s) {
   const int slices = a.d / kDnCols;
-  const size_t smem = sizeof(bf16) * kDnStages * kDnK * kDnRow;
+  const size_t smem = kDnStages * kDnStageBytes;
   cudaError_t e = cudaFuncSetAttribute(down_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int occ = 0;

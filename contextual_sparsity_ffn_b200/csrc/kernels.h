@@ -32,10 +32,6 @@ struct GateArgs {
   uint32_t* err;
 };
 cudaError_t launch_gate_compact(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
-// Same computation, warp-specialised and fed by bulk copies (gate_tma.cu); needs a ring of at least
-// four 2-row slots beside the staged tokens in shared memory.
-bool gate_tma_supported(int K, int B, int wdtype, bool x_f32);
-cudaError_t launch_gate_tma(const GateArgs& a, int wdtype, bool x_f32, int mode, cudaStream_t s);
 // Streaming version with an asynchronous compaction warp (gate_stream.cu); needs the staged tokens
 // to fit in shared memory.
 bool gate_stream_supported(int K, int B, int wdtype, bool x_f32);
