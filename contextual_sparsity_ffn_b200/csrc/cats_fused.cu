@@ -96,7 +96,9 @@ __device__ __forceinline__ void row_dot(const WT* __restrict__ row, const WT* __
 
 template <int NB> struct FusedGateU { static constexpr int value = NB <= 2 ? 16 : 8; };
 // Kept rows whose W_down^T slices are loaded together.
-template <int KD> struct FusedDownRows { static constexpr int value = KD <= 2 ? 4 : 2; };
+template <int NB, int KD> struct FusedDownRows {
+  static constexpr int value = NB * KD <= 2 ? 8 : (NB * KD <= 4 ? 4 : 2);  // a whole chunk at batch 1
+};
 
 // Tickets, drawn by thread 0.  Counter g hands out the chunks of block g, [lo(g), lo(g + 1)); a
 // counter found dry is flagged (word 1 of its line) and the thread moves on to the next counter
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr int EPV = Vec<WT>::N;
   constexpr int U = FusedGateU<NB>::value;
-  constexpr int DR = FusedDownRows<KD>::value;
+  constexpr int DR = FusedDownRows<NB, KD>::value;
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ int s_abort;
   __shared__ float s_v[2][kChunk][NB];

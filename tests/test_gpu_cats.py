@@ -340,3 +340,26 @@ def test_fused_decode_reglu_with_gate_bias():
         assert np.array_equal(got[~band], oracle.union_mask(oracle.cats_mask(a_ref, t))[~band])
         m = token_masks(idx, a_val, spec.h)
         assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= TOL_BF16_F32OUT
+
+
+def test_fused_decode_7b_low_threshold_keeps_negative_activations():
+    """t = 0.25 < max |SiLU| on the negative side (0.278): neurons with z in about (-2, -0.75)
+    are kept too, so the kept set is not one-sided; one-launch and two-call paths against the oracle."""
+    spec, x, _ = synth.llama2_7b_swiglu(0, n_eval=1, n_calib=1)
+    t = 0.25
+    a_ref = oracle.gate_activation(x, spec)
+    keep_ref = oracle.union_mask(oracle.cats_mask(a_ref, t))
+    assert (a_ref[0][keep_ref] < 0).sum() > 1000  # the case this test is for
+    layer = dev_layer(spec)
+    band = band_rows(a_ref, t)
+    for one_launch in (True, False):
+        if one_launch:
+            idx, a_val, out = run_fused(layer, x, t)
+        else:
+            idx, a_val, bufs = run_gate(layer, x, t)
+            out = run_sparse(layer, bufs)
+        got = np.zeros(spec.h, bool)
+        got[idx] = True
+        assert np.array_equal(got[~band], keep_ref[~band])
+        m = token_masks(idx, a_val, spec.h)
+        assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= TOL_BF16_F32OUT
