@@ -260,6 +260,78 @@ def dense_verify_measure(torch, cs, stream, K, W, world, dev):
             f"frac_of_{measured_hbm_gbs()[1]}_hbm": round(nbytes / (us_call * 1e-6) / 1e9 / measured_hbm_gbs()[0], 4)}
 
 
+def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
+    """SVD-predictor ReGLU workload (d 4096, h 11008, bf16, per-neuron thresholds at q = 0.9):
+    per step csffn_predict_lowrank, csffn_gate_mask on the predicted set (ReLU, t = 0) and
+    csffn_sparse_ffn_forward on the active set.  This step reads a few tens of MB, less than L2,
+    so L2 is flushed (a 256 MB write) before every step: step time = time of K x (flush + step)
+    minus time of K x flush, both as one CUDA graph.  The truncated SVD of W_gate is the offline
+    stage (outside the library), done here with torch on the device."""
+    spec, x, xc = synth.reglu_sparse(0, d=D, h=H, n_eval=N_TOKENS, n_calib=512)
+    layer = cs.FFNLayer.from_spec(spec, "cuda")
+    xs = cs.to_device(x, "cuda")
+    xcal = cs.to_device(xc, "cuda")
+    u, sv, vh = torch.linalg.svd(layer.w_gate.float().T, full_matrices=False)  # W_gate^T = U S V^T
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n = max(8, min(K, 50))
+    out_d = {}
+    for r in (256, 1024):
+        urt = (u[:, :r] * sv[:r]).T.contiguous().to(torch.bfloat16)
+        vr = vh[:r, :].T.contiguous().to(torch.bfloat16)
+        tau = torch.zeros(H, device=dev)
+        cs.calibrate_threshold(layer, xcal, 0.9, cs._abi.CAL_PER_NEURON_PRED, tau, u_rt=urt, v_r=vr)
+        ws = cs.new_workspace(layer, 1, r)
+        ci = torch.zeros(H, dtype=torch.int32, device=dev)
+        cc = torch.zeros(1, dtype=torch.int32, device=dev)
+        idx = torch.zeros(H, dtype=torch.int32, device=dev)
+        cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+        av = torch.zeros(1, H, device=dev)
+        o = torch.zeros(1, D, device=dev)
+
+        def step(k):
+            x1 = xs[k % N_TOKENS: k % N_TOKENS + 1]
+            cs.predict_lowrank(layer, x1, urt, vr, tau, ci, cc, ws)
+            cs.gate_mask(layer, x1, 0.0, idx, cnt, av, ws, cand_idx=ci, cand_count=cc)
+            cs.sparse_ffn_forward(layer, x1, idx, cnt, av, o, ws)
+
+        n_p, n_a = [], []
+        for k in range(min(n, N_TOKENS)):
+            step(k)
+            n_p.append(int(cc.item()))
+            n_a.append(int(cnt.item()))
+
+        def timed(with_step):
+            def f(k):
+                flush.zero_()
+                if with_step:
+                    step(k)
+            g = run_graph_steps(torch, f, n, 3, stream)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record()
+                g.replay()
+                e1.record()
+            torch.cuda.synchronize()
+            del g
+            return e0.elapsed_time(e1) * 1e3 / n
+
+        us = max_over_ranks(timed(True) - timed(False), world, dev)
+        mp, ma = float(np.mean(n_p)), float(np.mean(n_a))
+        nbytes = (r * D + H * r) * 2 + mp * D * 2 + 2 * ma * D * 2 + mp * 4 + ma * 8
+        out_d[f"r{r}"] = {"us_per_layer": round(us, 2), "predicted_rows": round(mp, 1), "active_rows": round(ma, 1),
+                          "bytes_needed_mb": round(nbytes / 1e6, 2),
+                          "achieved_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                          "launches_per_step": 5}
+        del ws
+    del flush, layer
+    torch.cuda.empty_cache()
+    out_d["path"] = ("csffn_predict_lowrank + csffn_gate_mask (predicted set) + csffn_sparse_ffn_forward; "
+                     "L2 flushed before every step")
+    return out_d
+
+
 def csffn_arm(args, world, rank, local):
     import torch
     from contextual_sparsity_ffn_b200 import binding as cs
@@ -413,6 +485,7 @@ def csffn_arm(args, world, rank, local):
                 detail[key]["speedup_vs_dense"] = round(u / detail[key]["us_per_layer"], 3)
         del g
         detail["dense_verify_70b_b16"] = dense_verify_measure(torch, cs, stream, K, W, world, dev)
+        detail["svd_reglu_q90"] = svd_reglu_measure(torch, cs, synth, stream, K, world, dev)
     del g_main
 
     # ---- end to end through the public API: pinned host x in, host out back, every step

@@ -9,7 +9,8 @@
 // and a statically partitioned stream ends in a long tail (CTAs with equal shares finished up to
 // 2.5x apart), so the rows are handed out dynamically in small chunks.
 //
-// Chunks of kChunk neuron rows come from ticket counters (one per contiguous block of chunks).
+// Chunks of kChunk neuron rows come from a ticket counter (in row order; the next ticket is drawn
+// one chunk ahead, so its round trip is hidden and 1.4 K draws per step do not contend).
 // The chunk's W_gate rows (contiguous) arrive in shared memory by one bulk copy issued while the
 // previous chunk is still being worked on, so every CTA keeps a chunk of gate rows in flight beside
 // its register loads.  For its chunk a CTA
@@ -36,7 +37,7 @@ namespace csffn {
 constexpr int kFusedThreads = 256;
 constexpr int kFusedWarps = kFusedThreads / kWarp;
 constexpr int kChunk = kFusedWarps;  // neuron rows per chunk, one per warp
-constexpr int kCounters = 32;        // ticket counters
+constexpr int kCounters = 1;         // ticket counters (one: measured faster than 4 or 32 blocks)
 constexpr int kCounterStride = 32;   // 32-bit words between counters (128 bytes)
 constexpr int kSumCols = 16;         // columns per slice of the final cross-CTA sum
 

@@ -14,8 +14,8 @@
 //
 // Down (down_mma_kernel): out[b, :] = sum_i v[b, i] W_down^T[i, :] with M = tokens, N = output
 // columns and K = neurons.  W_down^T rows and the matching slice of v are staged in shared memory
-// (cp.async, four-block ring, padded rows); W_down^T is read as B fragments by ldmatrix .trans and
-// v is split into bf16 high and low parts (two MMAs), so
+// (cp.async, four-block ring, padded rows); W_down^T is read as B fragments by ldmatrix .trans.
+// The gate/up epilogue stores v as bf16 high and low parts (two MMAs), so
 // the product carries about 16 mantissa bits of v.  Column tiles x neuron ranges, partials
 // summed by the last CTA of each column tile (in range order).
 #include "common.cuh"
@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kMmaThreads, 4) dense_gate_up_mma_kernel(const
   const bf16* Wg = reinterpret_cast<const bf16*>(p.W_gate);
   const bf16* Wu = reinterpret_cast<const bf16*>(p.W_up);
   const bf16* xg = reinterpret_cast<const bf16*>(p.x);
+  bf16* vhi = reinterpret_cast<bf16*>(p.v);  // [B, h] high parts, then [B, h] low parts
+  bf16* vlo = vhi + (size_t)B * h;
   const int n_ctiles = ((h + 15) / 16 + kMmaWarps - 1) / kMmaWarps;
   const int n_chunks = (d + kXChunk - 1) / kXChunk;
 
@@ -143,7 +145,13 @@ __global__ void __launch_bounds__(kMmaThreads, 4) dense_gate_up_mma_kernel(const
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int b = 8 * t + 2 * q + e;
-          if (b < B) p.v[(size_t)b * h + i] = gate_act(zg[t][2 * half + e] + beta, p.act) * zu[t][2 * half + e];
+          if (b < B) {
+            // v in two bf16 parts, hi = bf16(v) and lo = bf16(v - hi): the down MMAs take both
+            const float v = gate_act(zg[t][2 * half + e] + beta, p.act) * zu[t][2 * half + e];
+            const bf16 hi = __float2bfloat16_rn(v);
+            vhi[(size_t)b * h + i] = hi;
+            vlo[(size_t)b * h + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+          }
         }
     }
   }
@@ -160,23 +168,15 @@ constexpr int kDnCols = 64;
 constexpr int kDnK = 64;                    // neurons per staged block
 constexpr int kDnStages = 4;                // staged blocks (three in flight while one is used)
 constexpr int kDnRow = kDnCols + 8;         // W_down^T tile row stride in elements (144 B)
-constexpr int kVRow = kDnK + 8;             // v tile row stride in floats (conflict-free 8-byte reads)
+constexpr int kVRow = kDnK + 8;             // v tile row stride in bf16 (144 B: conflict-free 4-byte reads)
 constexpr size_t kDnWBytes = sizeof(bf16) * kDnK * kDnRow;
-constexpr size_t kDnStageBytes = kDnWBytes + sizeof(float) * 16 * kVRow;
+constexpr size_t kDnVBytes = sizeof(bf16) * 16 * kVRow;   // one part (hi or lo) of the v tile
+constexpr size_t kDnStageBytes = kDnWBytes + 2 * kDnVBytes;
 
 __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* smem_row) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
                : "=r"(r0), "=r"(r1)
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
-}
-
-// fp32 pair -> bf16x2 (round to nearest) and the bf16x2 of what that rounding left out
-__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
-  const float ra = a - __low2float(h2), rb = b - __high2float(h2);
-  const __nv_bfloat162 l2 = __floats2bfloat162_rn(ra, rb);
-  hi = *reinterpret_cast<const uint32_t*>(&h2);
-  lo = *reinterpret_cast<const uint32_t*>(&l2);
 }
 
 template <int NT>
@@ -194,12 +194,15 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
   const int k_lo = blk_lo * kDnK, k_hi = min(p.n_host, blk_hi * kDnK);
   const int n_blocks = blk_hi - blk_lo;
   auto w_tile = [&](int buf) { return reinterpret_cast<bf16*>(dn_smem + (size_t)buf * kDnStageBytes); };
-  auto v_tile = [&](int buf) { return reinterpret_cast<float*>(dn_smem + (size_t)buf * kDnStageBytes + kDnWBytes); };
+  // v tile of a stage: high parts [16][kVRow], then low parts [16][kVRow] (bf16)
+  auto v_tile = [&](int buf) { return reinterpret_cast<bf16*>(dn_smem + (size_t)buf * kDnStageBytes + kDnWBytes); };
+  const bf16* vhi = reinterpret_cast<const bf16*>(p.v);
+  const bf16* vlo = vhi + (size_t)B * h;
 
   // token rows B..15 of every staged v tile stay zero
-  for (int e = tid; e < kDnStages * 16 * kVRow; e += kMmaThreads) {
-    const int buf = e / (16 * kVRow), rem = e % (16 * kVRow);
-    if (rem / kVRow >= B) v_tile(buf)[rem] = 0.f;
+  for (int e = tid; e < kDnStages * 2 * 16 * kVRow; e += kMmaThreads) {
+    const int buf = e / (2 * 16 * kVRow), rem = e % (2 * 16 * kVRow);
+    if ((rem % (16 * kVRow)) / kVRow >= B) v_tile(buf)[rem] = __float2bfloat16_rn(0.f);
   }
   auto stage = [&](int blk, int buf) {  // neurons k_lo + 64 blk ..: W_down^T columns col0 .. col0 + 63, and v
     const int r0 = k_lo + blk * kDnK;
@@ -212,14 +215,15 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
       else
         *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
-    float* vt = v_tile(buf);
-    for (int e = tid; e < B * (kDnK / 4); e += kMmaThreads) {
-      const int b = e / (kDnK / 4), c = e % (kDnK / 4);
-      float* dst = vt + b * kVRow + c * 4;
-      if (r0 + c * 4 < k_hi)  // h % 4 == 0: a 4-neuron group is wholly in range or wholly out
-        cp_async16(dst, p.v + (size_t)b * h + r0 + c * 4, 0u);
+    bf16* vt = v_tile(buf);
+    for (int e = tid; e < 2 * B * (kDnK / 8); e += kMmaThreads) {
+      const int part = e / (B * (kDnK / 8)), rem = e % (B * (kDnK / 8));
+      const int b = rem / (kDnK / 8), c = rem % (kDnK / 8);
+      bf16* dst = vt + part * 16 * kVRow + b * kVRow + c * 8;
+      if (r0 + c * 8 < k_hi)  // h % 8 == 0: an 8-neuron group is wholly in range or wholly out
+        cp_async16(dst, (part ? vlo : vhi) + (size_t)b * h + r0 + c * 8, 0u);
       else
-        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
   };
@@ -242,19 +246,20 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
     cp_async_wait<kDnStages - 1>();
     __syncthreads();
     const bf16* wt = w_tile(buf);
-    const float* vt = v_tile(buf);
+    const bf16* vt = v_tile(buf);
 #pragma unroll
     for (int kk = 0; kk < kDnK; kk += 16) {
-      // A fragment (tokens x neurons) from the staged v: rows g and g + 8, neurons kk + 2q (+1, +8, +9)
-      const float2 v00 = *reinterpret_cast<const float2*>(vt + g * kVRow + kk + 2 * q);
-      const float2 v10 = *reinterpret_cast<const float2*>(vt + (g + 8) * kVRow + kk + 2 * q);
-      const float2 v01 = *reinterpret_cast<const float2*>(vt + g * kVRow + kk + 2 * q + 8);
-      const float2 v11 = *reinterpret_cast<const float2*>(vt + (g + 8) * kVRow + kk + 2 * q + 8);
+      // A fragments (tokens x neurons) of both parts of v: rows g and g + 8, neurons kk + 2q (+1, +8, +9)
       uint32_t ah[4], al[4];
-      split_bf16x2(v00.x, v00.y, ah[0], al[0]);  // row g, k 2q..2q+1
-      split_bf16x2(v10.x, v10.y, ah[1], al[1]);  // row g+8
-      split_bf16x2(v01.x, v01.y, ah[2], al[2]);  // row g, k 2q+8..
-      split_bf16x2(v11.x, v11.y, ah[3], al[3]);  // row g+8
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const bf16* vp = vt + part * 16 * kVRow;
+        uint32_t* a = part ? al : ah;
+        a[0] = *reinterpret_cast<const uint32_t*>(vp + g * kVRow + kk + 2 * q);            // row g, k 2q..
+        a[1] = *reinterpret_cast<const uint32_t*>(vp + (g + 8) * kVRow + kk + 2 * q);      // row g + 8
+        a[2] = *reinterpret_cast<const uint32_t*>(vp + g * kVRow + kk + 2 * q + 8);        // row g, k 2q + 8..
+        a[3] = *reinterpret_cast<const uint32_t*>(vp + (g + 8) * kVRow + kk + 2 * q + 8);  // row g + 8
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         // B fragment: neurons kk .. kk + 15 (rows of the staged block), columns 16 warp + 8 t ..
@@ -305,7 +310,7 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
 // ------------------------------------------------------------------------------------------
 bool dense_mma_supported(int d, int h, int B, int wdtype) {
   return wdtype == CSFFN_BF16 && B >= kDenseMmaMinBatch && B <= 16 && d % 128 == 0 && d % kDnCols == 0 &&
-         d / kDnCols <= kMaxSlices && h >= 16 && h % 4 == 0;
+         d / kDnCols <= kMaxSlices && h >= 16 && h % 8 == 0;
 }
 
 cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
