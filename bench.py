@@ -58,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--sparsity", type=float, default=0.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-detail", action="store_true", help="skip the 70%/90%/dense detail runs")
+    ap.add_argument("--only-dense-verify", action="store_true",
+                    help="time only the 70B-shaped 16-token dense verify (for profiling its kernels)")
     ap.add_argument("--rotate", type=int, default=8,
                     help="distinct layer weight sets the steps rotate over (8 keeps every step out of L2; "
                          "1 only for profiler captures, which flush caches themselves)")
@@ -262,8 +264,8 @@ def dense_verify_measure(torch, cs, stream, K, W, world, dev):
 
 def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
     """SVD-predictor ReGLU workload (d 4096, h 11008, bf16, per-neuron thresholds at q = 0.9):
-    per step csffn_predict_lowrank, csffn_gate_mask on the predicted set (ReLU, t = 0) and
-    csffn_sparse_ffn_forward on the active set.  This step reads a few tens of MB, less than L2,
+    per step csffn_predict_lowrank, then csffn_cats_ffn_forward on the predicted set (ReLU, t = 0:
+    gate on P, up and down on the active set, one launch).  This step reads a few tens of MB, less than L2,
     so L2 is flushed (a 256 MB write) before every step: step time = time of K x (flush + step)
     minus time of K x flush, both as one CUDA graph.  The truncated SVD of W_gate is the offline
     stage (outside the library), done here with torch on the device."""
@@ -291,8 +293,7 @@ def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
         def step(k):
             x1 = xs[k % N_TOKENS: k % N_TOKENS + 1]
             cs.predict_lowrank(layer, x1, urt, vr, tau, ci, cc, ws)
-            cs.gate_mask(layer, x1, 0.0, idx, cnt, av, ws, cand_idx=ci, cand_count=cc)
-            cs.sparse_ffn_forward(layer, x1, idx, cnt, av, o, ws)
+            cs.cats_ffn_forward(layer, x1, 0.0, idx, cnt, av, o, ws, cand_idx=ci, cand_count=cc)
 
         n_p, n_a = [], []
         for k in range(min(n, N_TOKENS)):
@@ -323,11 +324,11 @@ def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
         out_d[f"r{r}"] = {"us_per_layer": round(us, 2), "predicted_rows": round(mp, 1), "active_rows": round(ma, 1),
                           "bytes_needed_mb": round(nbytes / 1e6, 2),
                           "achieved_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
-                          "launches_per_step": 5}
+                          "launches_per_step": 3}
         del ws
     del flush, layer
     torch.cuda.empty_cache()
-    out_d["path"] = ("csffn_predict_lowrank + csffn_gate_mask (predicted set) + csffn_sparse_ffn_forward; "
+    out_d["path"] = ("csffn_predict_lowrank + csffn_cats_ffn_forward on the predicted set; "
                      "L2 flushed before every step")
     return out_d
 
@@ -548,22 +549,20 @@ def time_step_eager(torch, cs, layers, thr, xs, buf, out_t, stream, K):
 
 
 def e2e_measure(torch, cs, layers, thr, xs, buf, stream, K, W, world, dev):
-    """Same step through the public calls, with the token copied in from pinned host memory and the
-    output copied back to pinned host memory inside the timed region, every step."""
+    """Same step through the public C-ABI call that takes host buffers (csffn_cats_ffn_forward_host):
+    every step copies its token in from pinned host memory and its output back to pinned host memory
+    inside the timed region; the host waits for all K results at the end."""
     host_x = xs.cpu().pin_memory()
     host_out = torch.empty(K, D, dtype=torch.float32).pin_memory()
-    xd = torch.empty(1, D, dtype=torch.bfloat16, device=dev)
-    od = torch.empty(1, D, dtype=torch.float32, device=dev)
 
-    def step(k, dst):
+    def step(k):
         li = k % N_ROT
-        xd.copy_(host_x[k % N_TOKENS: k % N_TOKENS + 1], non_blocking=True)
-        cs.cats_decode(layers[li], xd, thr[li], od, buf)
-        dst.copy_(od[0], non_blocking=True)
+        cs.cats_ffn_forward_host(layers[li], host_x[k % N_TOKENS: k % N_TOKENS + 1], thr[li], buf.idx, buf.count,
+                                 buf.a_val, host_out[k % K: k % K + 1], buf.ws)
 
     with torch.cuda.stream(stream):
         for k in range(W):
-            step(k, host_out[k % K])
+            step(k)
     torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
@@ -571,13 +570,14 @@ def e2e_measure(torch, cs, layers, thr, xs, buf, stream, K, W, world, dev):
     t0 = time.perf_counter()
     with torch.cuda.stream(stream):
         for k in range(K):
-            step(k, host_out[k])
+            step(k)
     torch.cuda.synchronize()
     wall_ms = (time.perf_counter() - t0) * 1e3
     wall_ms = max_over_ranks(wall_ms, world, dev)
     return {"value": round(whole_job_us_per_layer(wall_ms, K, world), 3), "unit": UNIT,
             "h2d_bytes_per_step": 2 * D, "d2h_bytes_per_step": 4 * D,
-            "how": "eager calls through the binding; host wall clock around K steps incl. pinned H2D/D2H"}
+            "how": "csffn_cats_ffn_forward_host (one C-ABI call per step: pinned H2D of x, the kernel, "
+                   "D2H of out); host wall clock around K steps"}
 
 
 # ---------------------------------------------------------------------------------- oracle legs
@@ -657,6 +657,12 @@ def main(argv=None) -> int:
     world, rank, local = dist_env()
     if args.impl == "reference":
         res, rank = reference_arm(args, world, rank)
+    elif args.only_dense_verify:
+        import torch
+        from contextual_sparsity_ffn_b200 import binding as cs
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+        res = dense_verify_measure(torch, cs, torch.cuda.Stream(), args.steps, args.warmup, 1, dev)
     else:
         res, rank = csffn_arm(args, world, rank, local)
     if rank == 0 and res is not None:

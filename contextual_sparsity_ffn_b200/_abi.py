@@ -51,7 +51,8 @@ SIGNATURES = {
     "csffn_gate_mask": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "csffn_sparse_ffn_forward": (_I, [_L, _P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "csffn_dense_ffn_forward": (_I, [_L, _P, _I, _P, _I, _P, _Z, _P]),
-    "csffn_cats_ffn_forward": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _I, _P, _Z, _P]),
+    "csffn_cats_ffn_forward": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _P, _P, _I, _P, _Z, _P]),
+    "csffn_cats_ffn_forward_host": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "csffn_predict_lowrank": (_I, [_L, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "csffn_calibrate_workspace_size": (_Z, [_L, _I, _I, _I]),
     "csffn_calibrate_threshold": (_I, [_L, _P, _I, _F, _I, _P, _P, _I, _P, _P, _Z, _P]),

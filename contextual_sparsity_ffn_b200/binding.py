@@ -150,13 +150,36 @@ def sparse_ffn_forward(layer: FFNLayer, x: torch.Tensor, idx: torch.Tensor, coun
 
 def cats_ffn_forward(layer: FFNLayer, x: torch.Tensor, t: float, idx: torch.Tensor, count: torch.Tensor,
                      a_val: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, out_mode: Optional[int] = None,
+                     cand_idx: Optional[torch.Tensor] = None, cand_count: Optional[torch.Tensor] = None,
                      stream=None) -> None:
     B = x.shape[0] if x.dim() == 2 else 1
     if out_mode is None:
         out_mode = _abi.OUT_BF16 if out.dtype == torch.bfloat16 else _abi.OUT_F32
-    check(load().csffn_cats_ffn_forward(layer.ref(), _ptr(x), B, float(t), _ptr(idx), _ptr(count), _ptr(a_val),
-                                        _ptr(out), out_mode, _ptr(ws), _nbytes(ws), _stream(stream)),
+    check(load().csffn_cats_ffn_forward(layer.ref(), _ptr(x), B, float(t), _ptr(cand_idx), _ptr(cand_count),
+                                        _ptr(idx), _ptr(count), _ptr(a_val), _ptr(out), out_mode, _ptr(ws),
+                                        _nbytes(ws), _stream(stream)),
           "csffn_cats_ffn_forward")
+
+
+def _host_ptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("csffn host entry points take CPU tensors (pinned for asynchronous copies)")
+    if not t.is_contiguous():
+        raise ValueError("csffn takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def cats_ffn_forward_host(layer: FFNLayer, x_host: torch.Tensor, t: float, idx: torch.Tensor,
+                          count: torch.Tensor, a_val: torch.Tensor, out_host: torch.Tensor, ws: torch.Tensor,
+                          stream=None) -> None:
+    """csffn_cats_ffn_forward_host: x_host and out_host are CPU tensors (pinned memory keeps the
+    copies asynchronous); the result is in out_host once the stream has reached this call's copy."""
+    B = x_host.shape[0] if x_host.dim() == 2 else 1
+    out_mode = _abi.OUT_BF16 if out_host.dtype == torch.bfloat16 else _abi.OUT_F32
+    check(load().csffn_cats_ffn_forward_host(layer.ref(), _host_ptr(x_host), B, float(t), _ptr(idx), _ptr(count),
+                                             _ptr(a_val), _host_ptr(out_host), out_mode, _ptr(ws), _nbytes(ws),
+                                             _stream(stream)),
+          "csffn_cats_ffn_forward_host")
 
 
 def dense_ffn_forward(layer: FFNLayer, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,

@@ -204,6 +204,7 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
 }
 
 csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
+                                    const int32_t* cand_idx, const int32_t* cand_count,
                                     int32_t* idx, int32_t* count, float* a_val,
                                     void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
   csffn_status st = check_layer_shape(layer);
@@ -212,9 +213,10 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   if (out_mode != CSFFN_OUT_BF16 && out_mode != CSFFN_OUT_F32 && out_mode != CSFFN_OUT_F32_ACCUMULATE)
     return CSFFN_ERR_INVALID_ARG;
   if (!count) return CSFFN_ERR_INVALID_ARG;
+  if ((cand_idx == nullptr) != (cand_count == nullptr)) return CSFFN_ERR_INVALID_ARG;
   if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
   if (!cats_fused_supported(layer->d, B, layer->wdtype)) {
-    st = csffn_gate_mask(layer, x, B, t, nullptr, nullptr, idx, count, a_val, ws, ws_bytes, stream);
+    st = csffn_gate_mask(layer, x, B, t, cand_idx, cand_count, idx, count, a_val, ws, ws_bytes, stream);
     if (st != CSFFN_OK) return st;
     return csffn_sparse_ffn_forward(layer, x, B, idx, count, a_val, out, out_mode, ws, ws_bytes, stream);
   }
@@ -234,6 +236,8 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   a.bias = layer->gate_bias;
   a.t = t;
   a.act = layer->act;
+  a.cand_idx = cand_idx;
+  a.cand_count = cand_count;
   a.afull = at<float>(ws, L.afull);
   a.flags = at<uint8_t>(ws, L.flags);
   a.partial = at<float>(ws, L.partial);
@@ -247,6 +251,30 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   a.out = out;
   a.out_mode = out_mode;
   return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
+}
+
+csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,
+                                         int32_t* idx, int32_t* count, float* a_val,
+                                         void* out_host, int out_mode, void* ws, size_t ws_bytes, void* stream) {
+  csffn_status st = check_layer_shape(layer);
+  if (st != CSFFN_OK) return st;
+  if (B < 0 || B > CSFFN_MAX_BATCH) return CSFFN_ERR_INVALID_ARG;
+  if (out_mode != CSFFN_OUT_BF16 && out_mode != CSFFN_OUT_F32) return CSFFN_ERR_INVALID_ARG;
+  if (!count) return CSFFN_ERR_INVALID_ARG;
+  if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
+  if (!x_host || !out_host) return CSFFN_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(layer->d, layer->h, B, 0);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != CSFFN_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  void* xd = at<char>(ws, L.hx);
+  void* od = at<char>(ws, L.hout);
+  const size_t xbytes = (size_t)B * layer->d * esize(layer->wdtype);
+  const size_t obytes = (size_t)B * layer->d * (out_mode == CSFFN_OUT_BF16 ? 2 : 4);
+  if (cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return CSFFN_ERR_CUDA;
+  st = csffn_cats_ffn_forward(layer, xd, B, t, nullptr, nullptr, idx, count, a_val, od, out_mode, ws, ws_bytes,
+                              stream);
+  if (st != CSFFN_OK) return st;
+  return cuda_status(cudaMemcpyAsync(out_host, od, obytes, cudaMemcpyDeviceToHost, s));
 }
 
 csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,

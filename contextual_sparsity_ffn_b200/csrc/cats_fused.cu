@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   __shared__ int s_abort;
   __shared__ float s_v[2][kChunk][NB];
   __shared__ uint8_t s_keep[2][kChunk];
+  __shared__ int s_row[2][kChunk];  // neuron of each position of the chunk
   __shared__ int s_next[2];
   __shared__ uint32_t s_cnt[kFusedWarps];
   __shared__ float4 s_sum[kHalf / kWarp][4];
@@ -181,17 +182,31 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   const WT* Wd = reinterpret_cast<const WT*>(p.W_down_t);
   const uint32_t row_bytes = (uint32_t)(d * sizeof(WT));
 
+  // Rows are positions 0 .. n_rows - 1 of the candidate list (neuron cand_idx[j]) or, without one,
+  // the neurons themselves.  Keep flags and kept activations are stored by position.
+  const int32_t* cand = p.cand_idx;
+  const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
+  auto neuron = [&](int j) { return cand ? __ldg(cand + j) : j; };
+
   Tickets tk;
   tk.ctr = p.tickets;
-  tk.n_chunks = (h + kChunk - 1) / kChunk;
-  tk.G = tk.n_chunks < kCounters ? tk.n_chunks : kCounters;
+  tk.n_chunks = (n_rows + kChunk - 1) / kChunk;
+  tk.G = tk.n_chunks < kCounters ? (tk.n_chunks > 0 ? tk.n_chunks : 1) : kCounters;
   int g = blockIdx.x % tk.G;
   uint32_t t_pending = 0;  // thread 0: ticket drawn for the chunk after the one in flight
-  auto issue_gate = [&](int c) {  // thread 0: the chunk's W_gate rows -> gbuf, one bulk copy
-    const int r0 = c * kChunk;
-    const uint32_t bytes = (uint32_t)min(kChunk, h - r0) * row_bytes;
-    mbar_arrive_expect_tx(&s_bar, bytes);
-    bulk_load(gbuf, Wg + (size_t)r0 * d, bytes, &s_bar);
+  auto issue_gate = [&](int c) {  // thread 0: the chunk's W_gate rows -> gbuf (one copy, or one per row)
+    const int j0 = c * kChunk, n = min(kChunk, n_rows - j0);
+    mbar_arrive_expect_tx(&s_bar, (uint32_t)n * row_bytes);
+    if (!cand) {
+      bulk_load(gbuf, Wg + (size_t)j0 * d, (uint32_t)n * row_bytes, &s_bar);
+    } else {
+      int rows[kChunk];  // all indices fetched before the first copy, so their loads overlap
+#pragma unroll
+      for (int jj = 0; jj < kChunk; ++jj) rows[jj] = jj < n ? neuron(j0 + jj) : 0;
+#pragma unroll
+      for (int jj = 0; jj < kChunk; ++jj)
+        if (jj < n) bulk_load(gbuf + (size_t)jj * d, Wg + (size_t)rows[jj] * d, row_bytes, &s_bar);
+    }
   };
 
   if (tid == 0) {
@@ -220,14 +235,15 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   for (int it = 0; chunk >= 0; ++it) {
     const int buf = it & 1;
 
-    // 1. gate and threshold for row r (one per warp) from the prefetched rows
+    // 1. gate and threshold for position j (neuron r; one per warp) from the prefetched rows
     mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
-    const int r = chunk * kChunk + warp;
+    const int j = chunk * kChunk + warp;
+    const int r = j < n_rows ? neuron(j) : 0;
     float a[NB];
     bool any = false;
 #pragma unroll
     for (int b = 0; b < NB; ++b) a[b] = 0.f;
-    if (r < h) {
+    if (j < n_rows) {
       float z[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) z[b] = 0.f;
@@ -241,10 +257,10 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
         any |= kb;
       }
       if (lane == 0) {
-        p.flags[r] = any ? 1 : 0;
+        p.flags[j] = any ? 1 : 0;
 #pragma unroll
         for (int b = 0; b < NB; ++b)
-          if (b < B) p.afull[(size_t)b * h + r] = a[b];
+          if (b < B) p.afull[(size_t)b * h + j] = a[b];
       }
     }
     __syncthreads();  // gbuf is free: prefetch the next chunk's gate rows
@@ -274,6 +290,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
 #pragma unroll
       for (int b = 0; b < NB; ++b) s_v[buf][warp][b] = v[b];
       s_keep[buf][warp] = any ? 1 : 0;
+      s_row[buf][warp] = r;
     }
     __syncthreads();
 
@@ -282,7 +299,6 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
 #pragma unroll
     for (int j = 0; j < kChunk; ++j) m |= s_keep[buf][j] ? 1u << j : 0u;
     const int next = s_next[buf ^ 1];
-    const int row0 = chunk * kChunk;
     while (m) {
       int js[DR];
       uint4 w[DR][KD];
@@ -290,7 +306,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       for (int q = 0; q < DR; ++q) {
         js[q] = m ? __ffs(m) - 1 : -1;
         m &= m - 1u;
-        const WT* row = Wd + (size_t)(row0 + (js[q] < 0 ? 0 : js[q])) * d;
+        const WT* row = Wd + (size_t)s_row[buf][js[q] < 0 ? 0 : js[q]] * d;
 #pragma unroll
         for (int k = 0; k < KD; ++k) {
           const int c = lane + k * kWarp;
@@ -413,10 +429,11 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     }
   } else {
     // ------------------------------------------------------------ compaction of the active list
-    // CTA k owns the 32-row words [wa, wb); the kept rows before wa are counted from the flag
-    // bytes (each 0 or 1, so the popcount of a 32-bit word of flags counts its kept rows).
+    // CTA k owns the 32-position words [wa, wb); the kept positions before wa are counted from the
+    // flag bytes (each 0 or 1, so the popcount of a 32-bit word of flags counts its kept rows).
+    // Position j is written out as its neuron (ascending, as the candidate list is).
     const int ct = tid - kHalf, cw = warp - kHalf / kWarp;
-    const int n_words = (h + kWarp - 1) / kWarp;
+    const int n_words = (n_rows + kWarp - 1) / kWarp;
     const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
     const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
     if (wa < wb || blockIdx.x == gridDim.x - 1) {
@@ -435,12 +452,12 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       named_sync(2, kHalf);
       for (int w0 = wa; w0 < wb; w0 += kHalf / kWarp) {
         const int w = w0 + cw;
-        const int r = w * kWarp + lane;
-        const bool in = w < wb && r < h;
-        const bool f = in && __ldcg(p.flags + r) != 0;
+        const int jp = w * kWarp + lane;
+        const bool in = w < wb && jp < n_rows;
+        const bool f = in && __ldcg(p.flags + jp) != 0;
         float av[NB];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + r) : 0.f;
+        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
         const uint32_t m = __ballot_sync(0xffffffffu, f);
         if (lane == 0) s_cnt[cw] = __popc(m);
         named_sync(2, kHalf);
@@ -452,7 +469,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
         }
         if (f) {
           const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
-          p.idx[pos] = r;
+          p.idx[pos] = neuron(jp);
 #pragma unroll
           for (int b = 0; b < NB; ++b)
             if (b < B) p.a_val[(size_t)b * h + pos] = av[b];

@@ -47,6 +47,8 @@ struct WsLayout {
   size_t flags;      // uint8 [h]                      per-neuron keep flags (fused path)
   size_t partial;    // fp32 [partial_rows(max_batch)][d]
   size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
+  size_t hx;         // [max_batch][d] (4 B each)      tokens staged from host memory (host entry point)
+  size_t hout;       // fp32 [max_batch][d]            output staged for the copy back to host memory
   size_t total;
   int max_chunks;
 };
@@ -88,6 +90,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   o = align_up(o, 256);
   L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);
   o = align_up(o, 256);
+  L.hx = o;         o += align_up(sizeof(float) * (size_t)max_batch * d, 256);
+  L.hout = o;       o += align_up(sizeof(float) * (size_t)max_batch * d, 256);
   L.total = o;
   return L;
 }

@@ -118,8 +118,10 @@ struct FusedArgs {
   const float* bias;
   float t;
   int act;
-  float* afull;      // [B, h] scratch: kept activation per neuron
-  uint8_t* flags;    // [h] scratch: keep flag per neuron (16-byte aligned)
+  const int32_t* cand_idx;    // rows to consider (ascending neurons), or NULL = all h neurons
+  const int32_t* cand_count;  // device count of cand_idx
+  float* afull;      // [B, h] scratch: kept activation per row position
+  uint8_t* flags;    // [h] scratch: keep flag per row position (16-byte aligned)
   float* partial;    // [partial_rows / B][B, d] scratch: one fp32 partial of out per CTA
   int partial_rows;  // capacity of partial in rows of d floats
   int chunk_rows;    // neuron rows per chunk (set by the launcher)

@@ -153,11 +153,26 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
  * d % 128 == 0 (bf16; d % 64 for fp32) and the tokens fit in shared memory beside the weight
  * buffers; other shapes fall back to the two-call path inside this call.  The mask and a_val are
  * bit-for-bit repeatable; out may differ from launch to launch in the last bits (rows reach CTAs
- * dynamically, so the order of the final fp32 sum varies).  ws sized by csffn_workspace_size for
- * this layer and batch.  B == 0: writes *count = 0. */
+ * dynamically, so the order of the final fp32 sum varies).  cand_idx / cand_count (both or
+ * neither): as in csffn_gate_mask, only the listed neurons (ascending, device count) are
+ * considered, e.g. the set csffn_predict_lowrank predicts ([SVDP] Fig. 3: the gate runs on the
+ * predicted set; with act = RELU and t = 0 the kept set is {z > 0} within it).  ws sized by
+ * csffn_workspace_size for this layer and batch.  B == 0: writes *count = 0. */
 csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
+                                    const int32_t* cand_idx, const int32_t* cand_count,
                                     int32_t* idx, int32_t* count, float* a_val,
                                     void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* csffn_cats_ffn_forward with the tokens and the output in host memory: copies x_host [B, d]
+ * (weight dtype) into the workspace, runs the one-launch step, and copies out [B, d] (bf16 or fp32;
+ * out_mode CSFFN_OUT_BF16 or CSFFN_OUT_F32) back to out_host, all asynchronously on `stream`.
+ * idx, count and a_val stay in device memory as in csffn_cats_ffn_forward.  The host buffers must
+ * stay valid until the stream reaches the copies; page-locked (pinned) host memory keeps the
+ * copies asynchronous, pageable memory makes them synchronous.  ws sized by csffn_workspace_size
+ * for this layer and batch (it holds the staged tokens and output).  B == 0: writes *count = 0. */
+csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,
+                                         int32_t* idx, int32_t* count, float* a_val,
+                                         void* out_host, int out_mode, void* ws, size_t ws_bytes, void* stream);
 
 /* Dense gated FFN over all h neurons (the full model that verifies a chunk of
  * sparse-drafted tokens, [SIRIUS] "Approach"; also the speed-up baseline).

@@ -166,3 +166,59 @@ def test_predictor_full_rank_is_the_gate():
     got[P] = True
     clear = np.abs(z) > 0.05 * np.sqrt(np.mean(z * z))
     assert np.array_equal(got[clear], (z > 0)[clear])
+
+
+@pytest.mark.parametrize("d,h,r", [(1024, 2048, 128), (4096, 11008, 256)])
+@pytest.mark.parametrize("B", [1, 4])
+def test_predict_then_one_launch_step(d, h, r, B):
+    """csffn_predict_lowrank, then csffn_cats_ffn_forward on the predicted set (ReLU, t = 0): the same
+    active set as the gathered gate of the two-call path and the oracle's sequential ReGLU output."""
+    spec, x, xc, urt, vr, tau_ref = reglu_case(d, h, r, 512)
+    x = x[:B]
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, B, r)
+    tau = torch.from_numpy(tau_ref.astype(np.float32)).cuda()
+    ci = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xd = dev(x)
+    cs.predict_lowrank(layer, xd, dev(urt), dev(vr), tau, ci, cc, ws)
+    idx = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    av = torch.zeros(B, h, device="cuda")
+    out = torch.full((B, d), float("nan"), device="cuda")
+    cs.cats_ffn_forward(layer, xd, 0.0, idx, cnt, av, out, ws, cand_idx=ci, cand_count=cc)
+    assert cs.check_status(ws) == 0
+    n = int(cnt.item())
+    idx_f = idx[:n].cpu().numpy()
+    av_f = av[:, :n].cpu().numpy().astype(np.float64)
+    out_f = out.cpu().numpy().astype(np.float64)
+    assert_index_list(idx_f, h)
+    P = ci[:int(cc.item())].cpu().numpy()
+    assert set(idx_f.tolist()) <= set(P.tolist())
+    # the two-call path on the same predicted set
+    idx2, a_val2, bufs = run_gate(layer, x, 0.0, ws=ws, cand=(ci, cc))
+    z = oracle.gate_preactivation(x, spec)
+    zrms = np.sqrt(np.mean(z * z))
+    clear = (np.abs(z) > 1e-3 * zrms).all(axis=0)
+    g1, g2 = np.zeros(h, bool), np.zeros(h, bool)
+    g1[idx_f], g2[idx2] = True, True
+    assert np.array_equal(g1[clear], g2[clear])
+    amask = np.zeros((B, h), bool)
+    amask[:, idx_f] = av_f != 0.0
+    ref, _ = oracle.reglu_sequential(x, spec, amask)
+    assert oracle.rel_l2(out_f, ref) <= 1e-4
+
+
+def test_one_launch_step_empty_candidate_list():
+    spec, x, xc, urt, vr, tau_ref = reglu_case(1024, 2048, 128, 512)
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 1)
+    ci = torch.zeros(spec.h, dtype=torch.int32, device="cuda")
+    cc = torch.zeros(1, dtype=torch.int32, device="cuda")  # nothing predicted
+    idx = torch.zeros(spec.h, dtype=torch.int32, device="cuda")
+    cnt = torch.full((1,), 5, dtype=torch.int32, device="cuda")
+    av = torch.zeros(1, spec.h, device="cuda")
+    out = torch.full((1, spec.d), float("nan"), device="cuda")
+    cs.cats_ffn_forward(layer, dev(x[:1]), 0.0, idx, cnt, av, out, ws, cand_idx=ci, cand_count=cc)
+    assert cs.check_status(ws) == 0
+    assert int(cnt.item()) == 0 and torch.all(out == 0)

@@ -363,3 +363,25 @@ def test_fused_decode_7b_low_threshold_keeps_negative_activations():
         assert np.array_equal(got[~band], keep_ref[~band])
         m = token_masks(idx, a_val, spec.h)
         assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= TOL_BF16_F32OUT
+
+
+def test_fused_decode_host_buffers():
+    """csffn_cats_ffn_forward_host: tokens in and output out through pinned host memory give the
+    device entry point's result (bf16 and fp32 outputs)."""
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=64)
+    t = oracle.calibrate_global(xc, spec, 0.5)
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, 2)
+    idx_d, a_val_d, out_d = run_fused(layer, x, t, ws=ws)
+    xh = dev(x).cpu().pin_memory()
+    for dtype, tol in ((torch.float32, 1e-6), (torch.bfloat16, TOL_BF16)):
+        oh = torch.full((2, spec.d), float("nan"), dtype=dtype).pin_memory()
+        idx = torch.zeros(spec.h, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+        av = torch.zeros(2, spec.h, device="cuda")
+        cs.cats_ffn_forward_host(layer, xh, t, idx, cnt, av, oh, ws)
+        torch.cuda.synchronize()
+        assert cs.check_status(ws) == 0
+        n = int(cnt.item())
+        assert np.array_equal(idx[:n].cpu().numpy(), idx_d)
+        assert oracle.rel_l2(oh.float().numpy().astype(np.float64), out_d) <= tol
