@@ -18,8 +18,11 @@
 // The gate/up epilogue stores v as bf16 high and low parts (two MMAs), so
 // the product carries about 16 mantissa bits of v.  Column tiles x neuron ranges, partials
 // summed by the last CTA of each column tile (in range order).
+#include <cuda.h>  // CUtensorMap and its encoder's types (the encoder itself comes from the runtime)
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace csffn {
 
@@ -160,73 +163,83 @@ __global__ void __launch_bounds__(kMmaThreads, 4) dense_gate_up_mma_kernel(const
 // ------------------------------------------------------------------------------------------
 // Down: out[b, :] = sum_i v[b, i] * W_down^T[i, :] for i < h.
 // CTA tile: 64 output columns x a range of neurons; warp w owns columns 16 w .. 16 w + 15 (two
-// n tiles) for all 16 tokens.  W_down^T rows of the tile (128 B each) and the tokens' v for the same
-// neurons are staged 64 neurons at a time in a four-block cp.async ring, in rows padded so that
-// ldmatrix and the A-fragment reads are free of bank conflicts.
+// n tiles) for all 16 tokens.  Per 64-neuron block, two TMA tensor copies fill a stage of a
+// four-stage ring: the 64 x 64 W_down^T tile (2-D map over [h, d]) and the tokens' v for the same
+// neurons, both bf16 parts (3-D map over [2][B][h]; token rows past B arrive as zeros).  Both land
+// with the 128-byte swizzle (16-byte chunk c of a 128-byte row r sits at chunk c ^ (r mod 8)), which
+// the ldmatrix and A-fragment addresses undo, so the reads are free of bank conflicts.
 // ------------------------------------------------------------------------------------------
 constexpr int kDnCols = 64;
-constexpr int kDnK = 64;                    // neurons per staged block
-constexpr int kDnStages = 4;                // staged blocks (three in flight while one is used)
-constexpr int kDnRow = kDnCols + 8;         // W_down^T tile row stride in elements (144 B)
-constexpr int kVRow = kDnK + 8;             // v tile row stride in bf16 (144 B: conflict-free 4-byte reads)
-constexpr size_t kDnWBytes = sizeof(bf16) * kDnK * kDnRow;
-constexpr size_t kDnVBytes = sizeof(bf16) * 16 * kVRow;   // one part (hi or lo) of the v tile
-constexpr size_t kDnStageBytes = kDnWBytes + 2 * kDnVBytes;
+constexpr int kDnK = 64;                             // neurons per staged block
+constexpr int kDnStages = 4;                         // staged blocks (three in flight while one is used)
+constexpr uint32_t kDnWBytes = kDnK * kDnCols * 2;   // W_down^T tile: 64 rows of 128 B
+constexpr uint32_t kDnVBytes = 2 * 16 * kDnK * 2;    // v tile: [part][token] rows of 128 B
+constexpr uint32_t kDnStageBytes = kDnWBytes + kDnVBytes;  // 12 KB, a multiple of 1 KB
+
+// Byte offset of byte `col_byte` of row `row` in a tile of 128-byte rows written with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t col_byte) {
+  return row * 128u + ((((col_byte >> 4) ^ (row & 7u)) << 4) | (col_byte & 15u));
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 
 __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* smem_row) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
                : "=r"(r0), "=r"(r1)
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
 }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
-template <int NT>
-__global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs p, int ranges) {
-  extern __shared__ __align__(128) unsigned char dn_smem[];
+__global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs p, int ranges,
+                                                                  const __grid_constant__ CUtensorMap tm_w,
+                                                                  const __grid_constant__ CUtensorMap tm_v) {
+  extern __shared__ __align__(1024) unsigned char dn_smem_raw[];
+  __shared__ __align__(8) uint64_t s_bar[kDnStages];
+  __shared__ int s_abort;
   __shared__ bool s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, q = lane & 3;
-  const int d = p.d, h = p.h, B = p.B;
-  const bf16* Wd = reinterpret_cast<const bf16*>(p.W_down_t);
+  const int d = p.d, B = p.B;
+  // the swizzle pattern repeats every 1 KB: stage buffers start on a 1 KB boundary
+  unsigned char* dn_smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(dn_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int col0 = blockIdx.x * kDnCols;
   const int ry = blockIdx.y;
-  // neuron range of this CTA, in whole blocks (block starts stay 16-byte aligned in v)
+  // neuron range of this CTA, in whole 64-neuron blocks; rows past h arrive as zeros
   const int n_blk = (p.n_host + kDnK - 1) / kDnK;
   const int blk_lo = (int)((long long)n_blk * ry / ranges), blk_hi = (int)((long long)n_blk * (ry + 1) / ranges);
-  const int k_lo = blk_lo * kDnK, k_hi = min(p.n_host, blk_hi * kDnK);
+  const int k_lo = blk_lo * kDnK;
   const int n_blocks = blk_hi - blk_lo;
-  auto w_tile = [&](int buf) { return reinterpret_cast<bf16*>(dn_smem + (size_t)buf * kDnStageBytes); };
-  // v tile of a stage: high parts [16][kVRow], then low parts [16][kVRow] (bf16)
-  auto v_tile = [&](int buf) { return reinterpret_cast<bf16*>(dn_smem + (size_t)buf * kDnStageBytes + kDnWBytes); };
-  const bf16* vhi = reinterpret_cast<const bf16*>(p.v);
-  const bf16* vlo = vhi + (size_t)B * h;
 
-  // token rows B..15 of every staged v tile stay zero
-  for (int e = tid; e < kDnStages * 2 * 16 * kVRow; e += kMmaThreads) {
-    const int buf = e / (2 * 16 * kVRow), rem = e % (2 * 16 * kVRow);
-    if ((rem % (16 * kVRow)) / kVRow >= B) v_tile(buf)[rem] = __float2bfloat16_rn(0.f);
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < kDnStages; ++i) mbar_init(&s_bar[i], 1);
+    fence_mbar_init();
   }
-  auto stage = [&](int blk, int buf) {  // neurons k_lo + 64 blk ..: W_down^T columns col0 .. col0 + 63, and v
-    const int r0 = k_lo + blk * kDnK;
-    bf16* wt = w_tile(buf);
-    for (int e = tid; e < kDnK * (kDnCols / 8); e += kMmaThreads) {
-      const int rr = e >> 3, v = e & 7;
-      bf16* dst = wt + rr * kDnRow + v * 8;
-      if (r0 + rr < k_hi)
-        cp_async16(dst, Wd + (size_t)(r0 + rr) * d + col0 + v * 8, 0u);
-      else
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    bf16* vt = v_tile(buf);
-    for (int e = tid; e < 2 * B * (kDnK / 8); e += kMmaThreads) {
-      const int part = e / (B * (kDnK / 8)), rem = e % (B * (kDnK / 8));
-      const int b = rem / (kDnK / 8), c = rem % (kDnK / 8);
-      bf16* dst = vt + part * 16 * kVRow + b * kVRow + c * 8;
-      if (r0 + c * 8 < k_hi)  // h % 8 == 0: an 8-neuron group is wholly in range or wholly out
-        cp_async16(dst, (part ? vlo : vhi) + (size_t)b * h + r0 + c * 8, 0u);
-      else
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_commit();
+  __syncthreads();
+  auto issue = [&](int blk) {  // thread 0: block blk into its stage
+    const int buf = blk % kDnStages, r0 = k_lo + blk * kDnK;
+    unsigned char* st = dn_smem + (size_t)buf * kDnStageBytes;
+    mbar_arrive_expect_tx(&s_bar[buf], kDnStageBytes);
+    tma_load_2d(st, &tm_w, col0, r0, &s_bar[buf]);
+    tma_load_3d(st + kDnWBytes, &tm_v, r0, 0, 0, &s_bar[buf]);
   };
+  if (tid == 0)
+    for (int b0 = 0; b0 < kDnStages - 1 && b0 < n_blocks; ++b0) issue(b0);
 
   float acc[2][4];
 #pragma unroll
@@ -234,38 +247,36 @@ __global__ void __launch_bounds__(kMmaThreads, 4) down_mma_kernel(const DownArgs
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
 
-#pragma unroll
-  for (int s0 = 0; s0 < kDnStages - 1; ++s0) {
-    if (s0 < n_blocks) stage(s0, s0);
-    else cp_async_commit();  // empty group: every iteration waits on the same group count
-  }
   for (int blk = 0; blk < n_blocks; ++blk) {
+    // the stage of block blk - 1 is free (barrier at the end of the last iteration): refill it
+    if (tid == 0 && blk + kDnStages - 1 < n_blocks) {
+      fence_proxy_async_smem();
+      issue(blk + kDnStages - 1);
+    }
     const int buf = blk % kDnStages;
-    if (blk + kDnStages - 1 < n_blocks) stage(blk + kDnStages - 1, (blk + kDnStages - 1) % kDnStages);
-    else cp_async_commit();
-    cp_async_wait<kDnStages - 1>();
-    __syncthreads();
-    const bf16* wt = w_tile(buf);
-    const bf16* vt = v_tile(buf);
+    mbar_wait(&s_bar[buf], (uint32_t)((blk / kDnStages) & 1), p.err, &s_abort);
+    const unsigned char* wt = dn_smem + (size_t)buf * kDnStageBytes;
+    const unsigned char* vt = wt + kDnWBytes;
 #pragma unroll
     for (int kk = 0; kk < kDnK; kk += 16) {
       // A fragments (tokens x neurons) of both parts of v: rows g and g + 8, neurons kk + 2q (+1, +8, +9)
       uint32_t ah[4], al[4];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        const bf16* vp = vt + part * 16 * kVRow;
         uint32_t* a = part ? al : ah;
-        a[0] = *reinterpret_cast<const uint32_t*>(vp + g * kVRow + kk + 2 * q);            // row g, k 2q..
-        a[1] = *reinterpret_cast<const uint32_t*>(vp + (g + 8) * kVRow + kk + 2 * q);      // row g + 8
-        a[2] = *reinterpret_cast<const uint32_t*>(vp + g * kVRow + kk + 2 * q + 8);        // row g, k 2q + 8..
-        a[3] = *reinterpret_cast<const uint32_t*>(vp + (g + 8) * kVRow + kk + 2 * q + 8);  // row g + 8
+        const uint32_t r_lo = part * 16 + g, r_hi = part * 16 + g + 8;
+        const uint32_t c0 = (kk + 2 * q) * 2, c8 = (kk + 2 * q + 8) * 2;
+        a[0] = *reinterpret_cast<const uint32_t*>(vt + swz(r_lo, c0));
+        a[1] = *reinterpret_cast<const uint32_t*>(vt + swz(r_hi, c0));
+        a[2] = *reinterpret_cast<const uint32_t*>(vt + swz(r_lo, c8));
+        a[3] = *reinterpret_cast<const uint32_t*>(vt + swz(r_hi, c8));
       }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        // B fragment: neurons kk .. kk + 15 (rows of the staged block), columns 16 warp + 8 t ..
+        // B fragment: neurons kk .. kk + 15 (rows of the staged tile), columns 16 warp + 8 t ..
         uint32_t b0, b1;
-        const int lrow = kk + (lane & 15);
-        ldmatrix_x2_trans(b0, b1, wt + lrow * kDnRow + warp * 16 + t * 8);
+        const uint32_t lrow = kk + (lane & 15);
+        ldmatrix_x2_trans(b0, b1, wt + swz(lrow, (warp * 16 + t * 8) * 2));
         mma_16816(acc[t], ah[0], ah[1], ah[2], ah[3], b0, b1);
         mma_16816(acc[t], al[0], al[1], al[2], al[3], b0, b1);
       }
@@ -328,20 +339,57 @@ cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link against libcuda).
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static TensorMapEncodeFn tensor_map_encoder() {
+  static TensorMapEncodeFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<TensorMapEncodeFn>(nullptr);
+    return reinterpret_cast<TensorMapEncodeFn>(ptr);
+  }();
+  return fn;
+}
+
 cudaError_t launch_down_mma(const DownArgs& a, int max_ranges, cudaStream_t s) {
+  TensorMapEncodeFn encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  // W_down^T [h][d] bf16: boxes of 64 columns x 64 rows
+  CUtensorMap tm_w, tm_v;
+  const cuuint64_t wdim[2] = {(cuuint64_t)a.d, (cuuint64_t)a.h};
+  const cuuint64_t wstride[1] = {(cuuint64_t)a.d * 2};
+  const cuuint32_t wbox[2] = {kDnCols, kDnK};
+  const cuuint32_t ones[3] = {1, 1, 1};
+  if (encode(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.W_down_t), wdim, wstride, wbox, ones,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  // v as [2 parts][B][h] bf16: boxes of 64 neurons x 16 tokens x 2 parts
+  const cuuint64_t vdim[3] = {(cuuint64_t)a.h, (cuuint64_t)a.B, 2};
+  const cuuint64_t vstride[2] = {(cuuint64_t)a.h * 2, (cuuint64_t)a.B * a.h * 2};
+  const cuuint32_t vbox[3] = {kDnK, 16, 2};
+  if (encode(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<float*>(a.v), vdim, vstride, vbox, ones,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
   const int slices = a.d / kDnCols;
-  const size_t smem = kDnStages * kDnStageBytes;
-  cudaError_t e = cudaFuncSetAttribute(down_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = kDnStages * kDnStageBytes + 1024;  // + room to align the ring to 1 KB
+  cudaError_t e = cudaFuncSetAttribute(down_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, down_mma_kernel<2>, kMmaThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, down_mma_kernel, kMmaThreads, smem);
   if (e != cudaSuccess) return e;
   int ranges = sm_count() * (occ > 0 ? occ : 1) / slices;  // one wave
   if (ranges < 1) ranges = 1;
   if (ranges > max_ranges) ranges = max_ranges;
   if (ranges > (a.n_host + kDnK - 1) / kDnK) ranges = (a.n_host + kDnK - 1) / kDnK;
   dim3 grid(slices, ranges);
-  down_mma_kernel<2><<<grid, kMmaThreads, smem, s>>>(a, ranges);
+  down_mma_kernel<<<grid, kMmaThreads, smem, s>>>(a, ranges, tm_w, tm_v);
   return cudaGetLastError();
 }
 
