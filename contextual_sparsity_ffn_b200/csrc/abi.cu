@@ -253,6 +253,55 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
 }
 
+csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
+                                   const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
+                                   float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
+  csffn_status st = check_layer_shape(layer);
+  if (st != CSFFN_OK) return st;
+  if (B < 0 || B > CSFFN_MAX_BATCH) return CSFFN_ERR_INVALID_ARG;
+  if (out_mode != CSFFN_OUT_BF16 && out_mode != CSFFN_OUT_F32 && out_mode != CSFFN_OUT_F32_ACCUMULATE)
+    return CSFFN_ERR_INVALID_ARG;
+  if (!count) return CSFFN_ERR_INVALID_ARG;
+  if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
+  if (!x || !u_rt || !v_r || !tau || !idx || !a_val || !out || std::isnan(t)) return CSFFN_ERR_INVALID_ARG;
+  if (rank < 1 || rank > CSFFN_MAX_RANK) return CSFFN_ERR_INVALID_ARG;
+  if (rank % vec_elems(layer->wdtype) != 0) return CSFFN_ERR_ALIGNMENT;
+  if ((st = check_weights(layer, true, true, true)) != CSFFN_OK) return st;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(u_rt) || !aligned16(v_r)) return CSFFN_ERR_ALIGNMENT;
+  if (!cats_fused_supported(layer->d, B, layer->wdtype, rank)) return CSFFN_ERR_UNSUPPORTED_SHAPE;
+  const WsLayout L = ws_layout(layer->d, layer->h, B, rank);
+  if ((st = check_ws(ws, ws_bytes, L.hx)) != CSFFN_OK) return st;
+  FusedArgs a{};
+  a.W_gate = layer->w_gate;
+  a.W_up = layer->w_up;
+  a.W_down_t = layer->w_down_t;
+  a.x = x;
+  a.d = layer->d;
+  a.h = layer->h;
+  a.B = B;
+  a.bias = layer->gate_bias;
+  a.t = t;
+  a.act = layer->act;
+  a.u_rt = u_rt;
+  a.v_r = v_r;
+  a.tau = tau;
+  a.rank = rank;
+  a.ybuf = at<float>(ws, L.ybuf);
+  a.afull = at<float>(ws, L.afull);
+  a.flags = at<uint8_t>(ws, L.flags);
+  a.partial = at<float>(ws, L.partial);
+  a.partial_rows = partial_rows(B);
+  a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
+  a.tickets = at<uint32_t>(ws, L.tickets);
+  a.err = at<uint32_t>(ws, L.err);
+  a.idx = idx;
+  a.count = count;
+  a.a_val = a_val;
+  a.out = out;
+  a.out_mode = out_mode;
+  return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
+}
+
 csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,
                                          int32_t* idx, int32_t* count, float* a_val,
                                          void* out_host, int out_mode, void* ws, size_t ws_bytes, void* stream) {

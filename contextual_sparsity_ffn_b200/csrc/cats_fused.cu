@@ -44,6 +44,7 @@ constexpr int kSumCols = 16;         // columns per slice of the final cross-CTA
 // Fused control words (FusedArgs::ctl).
 constexpr int kCtlDone = 0;  // CTAs whose partials and flags are written
 constexpr int kCtlExit = 1;  // CTAs finished
+constexpr int kCtlY = 2;     // CTAs whose share of the predictor's y is written (predictor mode)
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
@@ -158,7 +159,31 @@ constexpr int kHalf = kFusedThreads / 2;            // threads of each end-phase
 constexpr int kSumRowsPar = kHalf / (kSumCols / 4);  // partials summed side by side
 constexpr int kSumLoads = (kFusedMaxCtas + kSumRowsPar - 1) / kSumRowsPar;
 
-template <typename WT, int NB, int KD>
+// acc[b] += row[0 .. n) . y_b[0 .. n): a row in shared memory against fp32 vectors y_b = ys + b * n.
+template <typename WT, int NB>
+__device__ __forceinline__ void smem_dot_f32(const WT* row, const float* ys, int n, int lane, float (&acc)[NB]) {
+  constexpr int EPV = Vec<WT>::N;
+  const int nv = n / EPV;
+#pragma unroll 4
+  for (int v = lane; v < nv; v += kWarp) {
+    float wf[EPV];
+    unpack(*reinterpret_cast<const uint4*>(row + (size_t)v * EPV), wf);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float yf[EPV];
+      load_x<EPV>(ys + (size_t)b * n + (size_t)v * EPV, yf);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) acc[b] = fmaf(wf[e], yf[e], acc[b]);
+    }
+  }
+}
+
+// PRED: predictor mode ("SVD Contextual Sparsity Predictors for Fast LLM Inference", Fig. 1 and
+// Fig. 3).  Before the chunk loop the grid computes y = x U_r (a warp per row of U_r^T) and meets
+// at a grid-wide count; the chunks then prefetch rows of V_r instead of W_gate, each warp forms
+// p = y . V_r[i] + beta_i, and only a neuron predicted by some token (p > tau_i) has its W_gate
+// row streamed and its activation thresholded; up and down follow as in the CATS mode.
+template <typename WT, int NB, int KD, bool PRED>
 __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const FusedArgs p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr int EPV = Vec<WT>::N;
@@ -176,11 +201,14 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   const int d = p.d, h = p.h, B = p.B;
   const int cpw = d / EPV / kFusedWarps;  // 16-byte columns of W_down^T owned by each warp
   WT* xs = reinterpret_cast<WT*>(smem_raw);
-  WT* gbuf = xs + (size_t)NB * d;  // W_gate rows of the current chunk [kChunk][d]
+  const int rowlen = PRED ? p.rank : d;  // elements of a prefetched row (V_r or W_gate)
+  WT* gbuf = xs + (size_t)NB * d;         // prefetched rows of the current chunk [kChunk][rowlen]
+  float* ys = reinterpret_cast<float*>(gbuf + (size_t)kChunk * rowlen);  // predictor mode: y [NB][rank]
   const WT* Wg = reinterpret_cast<const WT*>(p.W_gate);
   const WT* Wu = reinterpret_cast<const WT*>(p.W_up);
   const WT* Wd = reinterpret_cast<const WT*>(p.W_down_t);
-  const uint32_t row_bytes = (uint32_t)(d * sizeof(WT));
+  const uint32_t row_bytes = (uint32_t)(rowlen * sizeof(WT));
+  const WT* Wpre = PRED ? reinterpret_cast<const WT*>(p.v_r) : Wg;  // the rows the chunks prefetch
 
   // Rows are positions 0 .. n_rows - 1 of the candidate list (neuron cand_idx[j]) or, without one,
   // the neurons themselves.  Keep flags and kept activations are stored by position.
@@ -198,7 +226,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     const int j0 = c * kChunk, n = min(kChunk, n_rows - j0);
     mbar_arrive_expect_tx(&s_bar, (uint32_t)n * row_bytes);
     if (!cand) {
-      bulk_load(gbuf, Wg + (size_t)j0 * d, (uint32_t)n * row_bytes, &s_bar);
+      bulk_load(gbuf, Wpre + (size_t)j0 * rowlen, (uint32_t)n * row_bytes, &s_bar);
     } else {
       int rows[kChunk];  // all indices fetched before the first copy, so their loads overlap
 #pragma unroll
@@ -222,6 +250,32 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   }
   stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), B, d);
   __syncthreads();
+
+  if constexpr (PRED) {
+    // y[b][k] = x_b . U_r^T[k]: a warp per row, over the whole grid; then every CTA takes all of y
+    const WT* Urt = reinterpret_cast<const WT*>(p.u_rt);
+    const int rank = p.rank;
+    for (int k = blockIdx.x * kFusedWarps + warp; k < rank; k += gridDim.x * kFusedWarps) {
+      float yk[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) yk[b] = 0.f;
+      row_dot<WT, NB, FusedGateU<NB>::value>(Urt + (size_t)k * d, xs, d, lane, yk);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        yk[b] = warp_sum(yk[b]);
+        if (lane == 0 && b < B) __stcg(p.ybuf + (size_t)b * rank + k, yk[b]);
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      atomicAdd(&p.ctl[kCtlY], 1u);
+      wait_at_least(&p.ctl[kCtlY], gridDim.x, p.err);
+    }
+    __syncthreads();
+    for (int e = tid; e < NB * rank; e += kFusedThreads) ys[e] = e / rank < B ? __ldcg(p.ybuf + e) : 0.f;
+    __syncthreads();
+  }
 
   float acc[NB][KD][EPV];
 #pragma unroll
@@ -247,12 +301,28 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       float z[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) z[b] = 0.f;
-      smem_row_dot<WT, NB>(gbuf + (size_t)warp * d, xs, d, lane, z);
       const float beta = p.bias ? __ldg(p.bias + r) : 0.f;
+      bool gate_row = true;
+      if constexpr (PRED) {
+        // predictor: p = y . V_r[r] + beta against tau_r (union over tokens); the gate row streams
+        // from HBM only for a predicted neuron
+        smem_dot_f32<WT, NB>(gbuf + (size_t)warp * rowlen, ys, rowlen, lane, z);
+        const float tau = __ldg(p.tau + r);
+        bool pred = false;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          pred |= b < B && warp_sum(z[b]) + beta > tau;
+          z[b] = 0.f;
+        }
+        gate_row = pred;
+        if (pred) row_dot<WT, NB, FusedGateU<NB>::value>(Wg + (size_t)r * d, xs, d, lane, z);
+      } else {
+        smem_row_dot<WT, NB>(gbuf + (size_t)warp * d, xs, d, lane, z);
+      }
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const float ab = gate_act(warp_sum(z[b]) + beta, p.act);
-        const bool kb = b < B && fabsf(ab) > p.t;
+        const bool kb = gate_row && b < B && fabsf(ab) > p.t;
         a[b] = kb ? ab : 0.f;
         any |= kb;
       }
@@ -491,14 +561,19 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
         p.tickets[i * kCounterStride + 1] = 0u;
       }
       p.ctl[kCtlDone] = 0u;
+      p.ctl[kCtlY] = 0u;
       p.ctl[kCtlExit] = 0u;
       __threadfence();
     }
   }
 }
 
-// Dynamic shared memory: the staged tokens and one chunk of W_gate rows.
-static size_t fused_smem_bytes(int d, int nb, size_t es) { return (size_t)(nb + kChunk) * d * es; }
+// Dynamic shared memory: the staged tokens and one chunk of prefetched rows (W_gate, or V_r in
+// predictor mode, with the predictor's y beside them).
+static size_t fused_smem_bytes(int d, int nb, size_t es, int rank = 0) {
+  if (rank > 0) return (size_t)nb * d * es + (size_t)kChunk * rank * es + (size_t)nb * rank * sizeof(float);
+  return (size_t)(nb + kChunk) * d * es;
+}
 
 // Down-slice width per lane (16-byte columns) for a shape, 0 when the fused kernel does not take it.
 static int fused_kd(int d, int B, int wdtype) {
@@ -511,10 +586,10 @@ static int fused_kd(int d, int B, int wdtype) {
   return kd;
 }
 
-template <typename WT, int NB, int KD>
+template <typename WT, int NB, int KD, bool PRED>
 static cudaError_t fused_t(FusedArgs a, cudaStream_t s) {
-  auto kern = cats_fused_kernel<WT, NB, KD>;
-  const size_t smem = fused_smem_bytes(a.d, NB, sizeof(WT));
+  auto kern = cats_fused_kernel<WT, NB, KD, PRED>;
+  const size_t smem = fused_smem_bytes(a.d, NB, sizeof(WT), PRED ? a.rank : 0);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -540,39 +615,44 @@ static cudaError_t fused_t(FusedArgs a, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-bool cats_fused_supported(int d, int B, int wdtype) {
+bool cats_fused_supported(int d, int B, int wdtype, int rank) {
   const size_t es = wdtype == CSFFN_F32 ? 4 : 2;
   return B >= 1 && B <= kFusedMaxBatch && fused_smem_bytes(d, batch_tier(B), es) <= 200 * 1024 &&
-         fused_kd(d, B, wdtype) > 0;
+         fused_smem_bytes(d, batch_tier(B), es, rank) <= 200 * 1024 && fused_kd(d, B, wdtype) > 0;
 }
 
-template <typename WT, int NB>
+template <typename WT, int NB, bool PRED>
 static cudaError_t fused_kd_t(const FusedArgs& a, int kd, cudaStream_t s) {
   switch (kd) {
-    case 1: return fused_t<WT, NB, 1>(a, s);
-    case 2: return fused_t<WT, NB, 2>(a, s);
+    case 1: return fused_t<WT, NB, 1, PRED>(a, s);
+    case 2: return fused_t<WT, NB, 2, PRED>(a, s);
     default:
       if constexpr (Vec<WT>::N == 8 && NB > 1) return cudaErrorInvalidValue;  // rejected by fused_kd
-      else return fused_t<WT, NB, 4>(a, s);
+      else return fused_t<WT, NB, 4, PRED>(a, s);
+  }
+}
+
+template <bool PRED>
+static cudaError_t launch_fused_mode(const FusedArgs& a, int wdtype, int kd, cudaStream_t s) {
+  const int t = batch_tier(a.B);
+  if (wdtype == CSFFN_F32) {
+    switch (t) {
+      case 1: return fused_kd_t<float, 1, PRED>(a, kd, s);
+      case 2: return fused_kd_t<float, 2, PRED>(a, kd, s);
+      default: return fused_kd_t<float, 4, PRED>(a, kd, s);
+    }
+  }
+  switch (t) {
+    case 1: return fused_kd_t<bf16, 1, PRED>(a, kd, s);
+    case 2: return fused_kd_t<bf16, 2, PRED>(a, kd, s);
+    default: return fused_kd_t<bf16, 4, PRED>(a, kd, s);
   }
 }
 
 cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s) {
   const int kd = fused_kd(a.d, a.B, wdtype);
   if (kd == 0) return cudaErrorInvalidValue;
-  const int t = batch_tier(a.B);
-  if (wdtype == CSFFN_F32) {
-    switch (t) {
-      case 1: return fused_kd_t<float, 1>(a, kd, s);
-      case 2: return fused_kd_t<float, 2>(a, kd, s);
-      default: return fused_kd_t<float, 4>(a, kd, s);
-    }
-  }
-  switch (t) {
-    case 1: return fused_kd_t<bf16, 1>(a, kd, s);
-    case 2: return fused_kd_t<bf16, 2>(a, kd, s);
-    default: return fused_kd_t<bf16, 4>(a, kd, s);
-  }
+  return a.u_rt ? launch_fused_mode<true>(a, wdtype, kd, s) : launch_fused_mode<false>(a, wdtype, kd, s);
 }
 
 }  // namespace csffn

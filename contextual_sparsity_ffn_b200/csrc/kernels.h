@@ -120,6 +120,11 @@ struct FusedArgs {
   int act;
   const int32_t* cand_idx;    // rows to consider (ascending neurons), or NULL = all h neurons
   const int32_t* cand_count;  // device count of cand_idx
+  const void* u_rt;           // predictor mode (non-NULL): U_r^T [rank, d], V_r [h, rank], tau [h]
+  const void* v_r;
+  const float* tau;
+  int rank;
+  float* ybuf;                // [B, rank] scratch: y = x U_r
   float* afull;      // [B, h] scratch: kept activation per row position
   uint8_t* flags;    // [h] scratch: keep flag per row position (16-byte aligned)
   float* partial;    // [partial_rows / B][B, d] scratch: one fp32 partial of out per CTA
@@ -134,7 +139,7 @@ struct FusedArgs {
   void* out;
   int out_mode;
 };
-bool cats_fused_supported(int d, int B, int wdtype);
+bool cats_fused_supported(int d, int B, int wdtype, int rank = 0);
 cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
 
 // Radix selection and per-neuron selection (calibration).

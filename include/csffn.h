@@ -197,6 +197,21 @@ csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int 
                                    int32_t* cand_idx, int32_t* cand_count,
                                    void* ws, size_t ws_bytes, void* stream);
 
+/* The predictor pipeline of one decode step in a single kernel launch ([SVDP] Fig. 1 and Fig. 3):
+ * csffn_predict_lowrank followed by csffn_cats_ffn_forward on the predicted set computes the same.
+ *   y = x U_r; neuron i is predicted iff p[b,i] = y_b . V_r[i,:] + beta_i > tau[i] for some token b;
+ *   a predicted neuron's gate runs (z = x W_gate[i] + beta_i, a = act(z), token b keeps it iff
+ *   |a| > t: with act = RELU and t = 0, A = {z > 0} within the predicted set), and the kept rows'
+ *   up and down projections give out.  idx[0 .. *count) = ascending kept neurons, a_val as in
+ *   csffn_gate_mask, out as in csffn_sparse_ffn_forward.  The predicted set itself is not written.
+ *   u_rt [rank, d], v_r [h, rank] in layer->wdtype, rank % (8 for bf16, 4 for fp32) == 0.
+ *   Runs for the shapes csffn_cats_ffn_forward takes in one launch, with the rank's rows beside
+ *   them in shared memory; other shapes return CSFFN_ERR_UNSUPPORTED_SHAPE (use the two calls).
+ *   ws sized by csffn_workspace_size(layer, B, rank).  B == 0: writes *count = 0. */
+csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
+                                   const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
+                                   float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
 /* Workspace bytes for csffn_calibrate_threshold with n calibration vectors. */
 size_t csffn_calibrate_workspace_size(const csffn_layer* layer, int n, int mode, int rank);
 

@@ -222,3 +222,56 @@ def test_one_launch_step_empty_candidate_list():
     cs.cats_ffn_forward(layer, dev(x[:1]), 0.0, idx, cnt, av, out, ws, cand_idx=ci, cand_count=cc)
     assert cs.check_status(ws) == 0
     assert int(cnt.item()) == 0 and torch.all(out == 0)
+
+
+@pytest.mark.parametrize("d,h,r,B", [(1024, 2048, 128, 1), (1024, 2048, 128, 4), (4096, 11008, 256, 1),
+                                     (4096, 11008, 1024, 1), (4096, 11008, 256, 3)])
+def test_one_launch_svd_step(d, h, r, B):
+    """csffn_svd_ffn_forward (predictor, gate on the predicted set, up and down in one launch) against
+    the predictor + one-launch-on-candidates path and the oracle's sequential ReGLU."""
+    spec, x, xc, urt, vr, tau_ref = reglu_case(d, h, r, 512)
+    x = x[:B]
+    layer = dev_layer(spec)
+    ws = cs.new_workspace(layer, B, r)
+    tau = torch.from_numpy(tau_ref.astype(np.float32)).cuda()
+    xd, urt_d, vr_d = dev(x), dev(urt), dev(vr)
+    idx = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    av = torch.zeros(B, h, device="cuda")
+    out = torch.full((B, d), float("nan"), device="cuda")
+    cs.svd_ffn_forward(layer, xd, urt_d, vr_d, tau, 0.0, idx, cnt, av, out, ws)
+    assert cs.check_status(ws) == 0
+    n = int(cnt.item())
+    idx1 = idx[:n].cpu().numpy()
+    av1 = av[:, :n].cpu().numpy().astype(np.float64)
+    out1 = out.cpu().numpy().astype(np.float64)
+    assert_index_list(idx1, h)
+    # reference active set from the oracle, outside the predictor and gate bands
+    p = oracle.predict(x, urt, vr, spec.bias)
+    p_cal = oracle.predict(xc, urt, vr, spec.bias)
+    rms = np.sqrt(np.mean(p_cal * p_cal, axis=0))
+    tau64 = tau.cpu().numpy().astype(np.float64)
+    pred = oracle.union_mask(oracle.predicted_mask(p, tau64))
+    z = oracle.gate_preactivation(x, spec)
+    zrms = np.sqrt(np.mean(z * z))
+    active_ref = pred & (z > 0).any(axis=0)
+    clear = ~_pred_band(p, tau64, rms) & (np.abs(z) > 1e-3 * zrms).all(axis=0)
+    got = np.zeros(h, bool)
+    got[idx1] = True
+    assert np.array_equal(got[clear], active_ref[clear])
+    amask = np.zeros((B, h), bool)
+    amask[:, idx1] = av1 != 0.0
+    ref, _ = oracle.reglu_sequential(x, spec, amask)
+    assert oracle.rel_l2(out1, ref) <= 1e-4
+    # the same step as two calls (predictor, then the one-launch step on its candidates)
+    ci = torch.zeros(h, dtype=torch.int32, device="cuda")
+    cc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cs.predict_lowrank(layer, xd, urt_d, vr_d, tau, ci, cc, ws)
+    idx2 = torch.zeros(h, dtype=torch.int32, device="cuda")
+    cnt2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    av2 = torch.zeros(B, h, device="cuda")
+    out2 = torch.zeros(B, d, device="cuda")
+    cs.cats_ffn_forward(layer, xd, 0.0, idx2, cnt2, av2, out2, ws, cand_idx=ci, cand_count=cc)
+    got2 = np.zeros(h, bool)
+    got2[idx2[:int(cnt2.item())].cpu().numpy()] = True
+    assert np.array_equal(got[clear], got2[clear])
