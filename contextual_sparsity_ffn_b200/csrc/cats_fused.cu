@@ -12,16 +12,17 @@
 // Chunks of kChunk neuron rows come from a ticket counter (in row order; the next ticket is drawn
 // one chunk ahead, so its round trip is hidden and 1.4 K draws per step do not contend).
 // The chunk's W_gate rows (contiguous) arrive in shared memory by one bulk copy issued while the
-// previous chunk is still being worked on, so every CTA keeps a chunk of gate rows in flight beside
-// its register loads.  For its chunk a CTA
-//   1. has warp w reduce gate row r = chunk row w against the tokens (both in shared memory), add
-//      the bias, apply the activation and the threshold per token, and record the keep flag and
-//      the kept activations; then (block barrier, gate buffer free) thread 0 issues the next
-//      chunk's bulk copy;
-//   2. has the warp of a kept row stream W_up[r] from HBM and form v[b] = a[b] * u[b];
-//   3. (block barrier) streams the kept rows of W_down^T: warp w owns a fixed 1/8 of the d output
-//      columns and accumulates v[b] * W_down^T[r, its columns] in registers over all its chunks,
-//      so no atomics and no cross-warp traffic are needed until the end.
+// previous chunk is still being worked on.  For its chunk a CTA
+//   1. has warp w reduce gate row w against the tokens (both in shared memory), add the bias,
+//      apply the activation and the threshold per token, and record the keep flag and the kept
+//      activations; after one block barrier thread 0 issues the next chunk's bulk copy;
+//   2. appends the chunk's kept rows to a ring queue in shared memory.  Whenever 8 rows are
+//      queued (and for the rest after the CTA's last chunk) it flushes them: warp w streams W_up of
+//      queued row w from HBM and forms v[b] = a[b] * u[b]; after a barrier each warp streams its
+//      fixed 1/8 of the columns of the 8 W_down^T rows and accumulates v[b] * W_down^T[r, cols] in
+//      registers over all its batches (no atomics, no cross-warp traffic until the end).
+// So the up and down round trips are paid once per 8 kept rows, not once per chunk: at high
+// sparsity the chunk loop is a gate stream.
 // When the tickets run out each CTA writes its register partial of out (fp32 [B, d]).  After a
 // grid-wide count (all CTAs are co-resident: cooperative launch) half of each CTA's warps sum the
 // partials in 16-column slices while the other half compact the active list from the keep flags:
@@ -37,6 +38,8 @@ namespace csffn {
 constexpr int kFusedThreads = 256;
 constexpr int kFusedWarps = kFusedThreads / kWarp;
 constexpr int kChunk = kFusedWarps;  // neuron rows per chunk, one per warp
+constexpr int kQueueBatch = kFusedWarps;      // kept rows per up/down batch, one W_up row per warp
+constexpr int kQueueSlots = 2 * kQueueBatch;  // ring of queued kept rows (a chunk adds at most kChunk)
 constexpr int kCounters = 1;         // ticket counters (one: measured faster than 4 or 32 blocks)
 constexpr int kCounterStride = 32;   // 32-bit words between counters (128 bytes)
 constexpr int kSumCols = 16;         // columns per slice of the final cross-CTA sum
@@ -191,9 +194,11 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   constexpr int DR = FusedDownRows<NB, KD>::value;
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ int s_abort;
-  __shared__ float s_v[2][kChunk][NB];
-  __shared__ uint8_t s_keep[2][kChunk];
-  __shared__ int s_row[2][kChunk];  // neuron of each position of the chunk
+  __shared__ float s_v[kQueueBatch][NB];        // v of the batch being flushed
+  __shared__ int s_drow[kQueueBatch];            // its neurons
+  __shared__ uint8_t s_keep[2][kChunk];          // keep flags of the chunk (by parity)
+  __shared__ int s_qrow[kQueueSlots];            // queued kept rows: neuron
+  __shared__ float s_qa[kQueueSlots][NB];        // and kept activations per token
   __shared__ int s_next[2];
   __shared__ uint32_t s_cnt[kFusedWarps];
   __shared__ float4 s_sum[kHalf / kWarp][4];
@@ -285,6 +290,67 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
 #pragma unroll
       for (int e = 0; e < EPV; ++e) acc[b][k][e] = 0.f;
 
+  // Kept rows wait in a ring of kQueueSlots entries (neuron, kept activations); q_head / q_tail are
+  // the same in every thread.  flush(n) runs up and down for the n oldest entries: warp w streams
+  // W_up of entry w and forms v, then every warp streams its columns of the n W_down^T rows.
+  int q_head = 0, q_tail = 0;
+  auto flush = [&](int n) {
+    __syncthreads();  // queued entries are visible; the last batch's v and rows are no longer read
+    float v[NB];
+    int r = 0;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) v[b] = 0.f;
+    if (warp < n) {
+      const int slot = (q_head + warp) & (kQueueSlots - 1);
+      r = s_qrow[slot];
+      float u[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) u[b] = 0.f;
+      row_dot<WT, NB, U>(Wu + (size_t)r * d, xs, d, lane, u);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) v[b] = s_qa[slot][b] * warp_sum(u[b]);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) s_v[warp][b] = v[b];
+      s_drow[warp] = r;
+    }
+    __syncthreads();
+    uint32_t m = (1u << n) - 1u;
+    while (m) {
+      int js[DR];
+      uint4 w[DR][KD];
+#pragma unroll
+      for (int q = 0; q < DR; ++q) {
+        js[q] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1u;
+        const WT* row = Wd + (size_t)s_drow[js[q] < 0 ? 0 : js[q]] * d;
+#pragma unroll
+        for (int k = 0; k < KD; ++k) {
+          const int c = lane + k * kWarp;
+          w[q][k] = (js[q] >= 0 && c < cpw) ? ld_stream(row + (size_t)(warp * cpw + c) * EPV)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < DR; ++q) {
+        if (js[q] < 0) continue;
+#pragma unroll
+        for (int k = 0; k < KD; ++k) {
+          float wf[EPV];
+          unpack(w[q][k], wf);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float vb = s_v[js[q]][b];
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) acc[b][k][e] = fmaf(vb, wf[e], acc[b][k][e]);
+          }
+        }
+      }
+    }
+    q_head += n;
+  };
+
   int chunk = s_next[0];
   for (int it = 0; chunk >= 0; ++it) {
     const int buf = it & 1;
@@ -333,73 +399,33 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
           if (b < B) p.afull[(size_t)b * h + j] = a[b];
       }
     }
-    __syncthreads();  // gbuf is free: prefetch the next chunk's gate rows
+    if (lane == 0) s_keep[buf][warp] = any ? 1 : 0;
+    int cn = -1;
     if (tid == 0) {
-      const int cn = tk.resolve(g, t_pending);
+      cn = tk.resolve(g, t_pending);  // drawn a chunk ago: its round trip is over
       s_next[buf ^ 1] = cn;
-      if (cn >= 0) {
-        fence_proxy_async_smem();
-        issue_gate(cn);
-        t_pending = tk.draw(g);
-      }
+    }
+    __syncthreads();  // keep flags and the next chunk are visible; gbuf is free
+    if (tid == 0 && cn >= 0) {
+      fence_proxy_async_smem();
+      issue_gate(cn);  // prefetch the next chunk's rows
+      t_pending = tk.draw(g);
     }
 
-    // 2. up for a kept row, straight from HBM
-    float v[NB];
+    // 2. queue the chunk's kept rows; up and down run on batches of kQueueBatch queued rows
+    uint32_t mask = 0;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) v[b] = 0.f;
-    if (any) {
-      float u[NB];
+    for (int jj = 0; jj < kChunk; ++jj) mask |= s_keep[buf][jj] ? 1u << jj : 0u;
+    if (any && lane == 0) {
+      const int slot = (q_tail + __popc(mask & ((1u << warp) - 1u))) & (kQueueSlots - 1);
+      s_qrow[slot] = r;
 #pragma unroll
-      for (int b = 0; b < NB; ++b) u[b] = 0.f;
-      row_dot<WT, NB, U>(Wu + (size_t)r * d, xs, d, lane, u);
-#pragma unroll
-      for (int b = 0; b < NB; ++b) v[b] = a[b] * warp_sum(u[b]);
+      for (int b = 0; b < NB; ++b) s_qa[slot][b] = a[b];
     }
-    if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < NB; ++b) s_v[buf][warp][b] = v[b];
-      s_keep[buf][warp] = any ? 1 : 0;
-      s_row[buf][warp] = r;
-    }
-    __syncthreads();
-
-    // 3. kept rows of W_down^T, this warp's columns
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < kChunk; ++j) m |= s_keep[buf][j] ? 1u << j : 0u;
+    q_tail += __popc(mask);
     const int next = s_next[buf ^ 1];
-    while (m) {
-      int js[DR];
-      uint4 w[DR][KD];
-#pragma unroll
-      for (int q = 0; q < DR; ++q) {
-        js[q] = m ? __ffs(m) - 1 : -1;
-        m &= m - 1u;
-        const WT* row = Wd + (size_t)s_row[buf][js[q] < 0 ? 0 : js[q]] * d;
-#pragma unroll
-        for (int k = 0; k < KD; ++k) {
-          const int c = lane + k * kWarp;
-          w[q][k] = (js[q] >= 0 && c < cpw) ? ld_stream(row + (size_t)(warp * cpw + c) * EPV)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < DR; ++q) {
-        if (js[q] < 0) continue;
-#pragma unroll
-        for (int k = 0; k < KD; ++k) {
-          float wf[EPV];
-          unpack(w[q][k], wf);
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const float vb = s_v[buf][js[q]][b];
-#pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[b][k][e] = fmaf(vb, wf[e], acc[b][k][e]);
-          }
-        }
-      }
-    }
+    if (q_tail - q_head >= kQueueBatch) flush(kQueueBatch);
+    if (next < 0 && q_tail > q_head) flush(q_tail - q_head);  // this CTA's last chunk: drain
     chunk = next;
   }
 
