@@ -240,8 +240,7 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   a.cand_count = cand_count;
   a.afull = at<float>(ws, L.afull);
   a.flags = at<uint8_t>(ws, L.flags);
-  a.partial = at<float>(ws, L.partial);
-  a.partial_rows = partial_rows(B);
+  a.facc = at<float>(ws, L.facc);
   a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
   a.tickets = at<uint32_t>(ws, L.tickets);
   a.err = at<uint32_t>(ws, L.err);
@@ -289,8 +288,7 @@ csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int 
   a.ybuf = at<float>(ws, L.ybuf);
   a.afull = at<float>(ws, L.afull);
   a.flags = at<uint8_t>(ws, L.flags);
-  a.partial = at<float>(ws, L.partial);
-  a.partial_rows = partial_rows(B);
+  a.facc = at<float>(ws, L.facc);
   a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
   a.tickets = at<uint32_t>(ws, L.tickets);
   a.err = at<uint32_t>(ws, L.err);

@@ -9,8 +9,9 @@
 // and a statically partitioned stream ends in a long tail (CTAs with equal shares finished up to
 // 2.5x apart), so the rows are handed out dynamically in small chunks.
 //
-// Chunks of kChunk neuron rows come from a ticket counter (in row order; the next ticket is drawn
-// one chunk ahead, so its round trip is hidden and 1.4 K draws per step do not contend).
+// Chunks of kChunk neuron rows (kTailChunk at the end of the range) go to CTA b first (chunk b,
+// no draw), then come from a ticket counter in row order; the next ticket is drawn one chunk
+// ahead, so its round trip is hidden and 1.4 K draws per step do not contend.
 // The chunk's W_gate rows (contiguous) arrive in shared memory by one bulk copy issued while the
 // previous chunk is still being worked on.  For its chunk a CTA
 //   1. has warp w reduce gate row w against the tokens (both in shared memory), add the bias,
@@ -23,11 +24,14 @@
 //      registers over all its batches (no atomics, no cross-warp traffic until the end).
 // So the up and down round trips are paid once per 8 kept rows, not once per chunk: at high
 // sparsity the chunk loop is a gate stream.
-// When the tickets run out each CTA writes its register partial of out (fp32 [B, d]).  After a
-// grid-wide count (all CTAs are co-resident: cooperative launch) half of each CTA's warps sum the
-// partials in 16-column slices while the other half compact the active list from the keep flags:
-// CTA k takes a fixed range of 32-row words, counts the flags before it, and writes idx / a_val in
-// ascending neuron order.  Every wait is bounded; the last CTA out resets the counters.
+// When the tickets run out each CTA adds its register partial of out (fp32 [B, d]) into one of a
+// few accumulators in L2 by vector reductions, so the CTAs that finish early do so while the rest
+// are still streaming.  After one grid-wide meeting (all CTAs are co-resident: cooperative launch)
+// half of each CTA's warps turn an equal share of the accumulators into out and clear it, while
+// the other half compact the active list from the keep flags: CTA k takes a fixed range of 32-row
+// words, counts the flags before it, and writes idx / a_val in ascending neuron order.  Every wait
+// is bounded; the counters return to zero by themselves (the ticket counter is cleared by the
+// last CTA to arrive at the meeting).
 #include "common.cuh"
 #include "gemv.cuh"
 #include "kernels.h"
@@ -42,17 +46,36 @@ constexpr int kQueueBatch = kFusedWarps;      // kept rows per up/down batch, on
 constexpr int kQueueSlots = 2 * kQueueBatch;  // ring of queued kept rows (a chunk adds at most kChunk)
 constexpr int kCounters = 1;         // ticket counters (one: measured faster than 4 or 32 blocks)
 constexpr int kCounterStride = 32;   // 32-bit words between counters (128 bytes)
-constexpr int kSumCols = 16;         // columns per slice of the final cross-CTA sum
+constexpr int kTailChunk = 4;        // rows per chunk at the end of the row range
+constexpr int kTailGrids = 2;        // the last kTailGrids * grid chunks are of kTailChunk rows
 
 // Fused control words (FusedArgs::ctl).
-constexpr int kCtlDone = 0;  // CTAs whose partials and flags are written
-constexpr int kCtlExit = 1;  // CTAs finished
+constexpr int kCtlDone = 0;  // CTAs whose partial sums and flags are written (wraps to 0 on the last)
 constexpr int kCtlY = 2;     // CTAs whose share of the predictor's y is written (predictor mode)
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+// out[0..3] += (a, b, c, e) as one vector reduction in L2 (no return value); 16-byte aligned.
+__device__ __forceinline__ void red_add_v4(float* out, float a, float b, float c, float e) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(e)
+               : "memory");
+}
+
+// Bounded wait until *p == 0 (acquire).  Gives up after a second and records the timeout.
+__device__ __forceinline__ void wait_zero(const uint32_t* p, uint32_t* err) {
+  if (ld_acquire_u32(p) == 0u) return;
+  const uint64_t t0 = globaltimer_now();
+  while (ld_acquire_u32(p) != 0u) {
+    if (globaltimer_now() - t0 > 1000000000ull) {
+      atomicOr(err, kDevErrTimeout);
+      return;
+    }
+    __nanosleep(64);
+  }
 }
 
 // Bounded wait until *p >= target (acquire).  Gives up after a second and records the timeout.
@@ -105,18 +128,41 @@ template <int NB, int KD> struct FusedDownRows {
   static constexpr int value = NB * KD <= 2 ? 8 : (NB * KD <= 4 ? 4 : 2);  // a whole chunk at batch 1
 };
 
-// Tickets, drawn by thread 0.  Counter g hands out the chunks of block g, [lo(g), lo(g + 1)); a
-// counter found dry is flagged (word 1 of its line) and the thread moves on to the next counter
-// not flagged.  resolve() returns -1 once every counter is dry.
+// Chunks in row order: kChunk rows each, then (for the last kTailGrids grid widths of chunks)
+// kTailChunk rows each, so the work a CTA still holds when the tickets run out is small and the
+// CTAs finish close together.
+struct ChunkMap {
+  int n_rows, n_big, n_chunks;
+  __device__ void init(int rows, int grid) {
+    n_rows = rows;
+    const int tail = kTailGrids * grid * kTailChunk;  // rows wanted in small chunks
+    n_big = rows > tail ? (rows - tail) / kChunk : 0;
+    n_chunks = n_big + (rows - n_big * kChunk + kTailChunk - 1) / kTailChunk;
+  }
+  __device__ void rows(int c, int& j0, int& n) const {
+    if (c < n_big) {
+      j0 = c * kChunk;
+      n = kChunk;
+    } else {
+      j0 = n_big * kChunk + (c - n_big) * kTailChunk;
+      n = min(kTailChunk, n_rows - j0);
+    }
+  }
+};
+
+// Tickets, drawn by thread 0, for the chunks after the first grid width (CTA b starts on chunk b
+// without a draw).  Counter g hands out chunks base + [lo(g), lo(g + 1)); a counter found dry is
+// flagged (word 1 of its line) and the thread moves on to the next counter not flagged.
+// resolve() returns -1 once every counter is dry.
 struct Tickets {
   uint32_t* ctr;
-  int n_chunks, G;
+  int base, n_chunks, G;
   __device__ int lo(int g) const { return (int)((long long)n_chunks * g / G); }
   __device__ uint32_t draw(int g) const { return atomicAdd(ctr + g * kCounterStride, 1u); }
   __device__ int resolve(int& g, uint32_t t) const {
     for (;;) {
       const int c = lo(g) + (int)t;
-      if (c < lo(g + 1)) return c;
+      if (c < lo(g + 1)) return base + c;
       ctr[g * kCounterStride + 1] = 1u;
       uint32_t live = 0;  // bit i: counter i not flagged dry
 #pragma unroll
@@ -158,9 +204,8 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-constexpr int kHalf = kFusedThreads / 2;            // threads of each end-phase group
-constexpr int kSumRowsPar = kHalf / (kSumCols / 4);  // partials summed side by side
-constexpr int kSumLoads = (kFusedMaxCtas + kSumRowsPar - 1) / kSumRowsPar;
+constexpr int kHalf = kFusedThreads / 2;  // threads of each end-phase group
+constexpr int kCountLoads = 16;           // 16-byte flag loads in flight per thread (compaction)
 
 // acc[b] += row[0 .. n) . y_b[0 .. n): a row in shared memory against fp32 vectors y_b = ys + b * n.
 template <typename WT, int NB>
@@ -201,7 +246,6 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   __shared__ float s_qa[kQueueSlots][NB];        // and kept activations per token
   __shared__ int s_next[2];
   __shared__ uint32_t s_cnt[kFusedWarps];
-  __shared__ float4 s_sum[kHalf / kWarp][4];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = p.d, h = p.h, B = p.B;
   const int cpw = d / EPV / kFusedWarps;  // 16-byte columns of W_down^T owned by each warp
@@ -221,14 +265,18 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
   auto neuron = [&](int j) { return cand ? __ldg(cand + j) : j; };
 
+  ChunkMap cm;
+  cm.init(n_rows, (int)gridDim.x);
   Tickets tk;
   tk.ctr = p.tickets;
-  tk.n_chunks = (n_rows + kChunk - 1) / kChunk;
+  tk.base = min((int)gridDim.x, cm.n_chunks);
+  tk.n_chunks = cm.n_chunks - tk.base;
   tk.G = tk.n_chunks < kCounters ? (tk.n_chunks > 0 ? tk.n_chunks : 1) : kCounters;
   int g = blockIdx.x % tk.G;
   uint32_t t_pending = 0;  // thread 0: ticket drawn for the chunk after the one in flight
   auto issue_gate = [&](int c) {  // thread 0: the chunk's W_gate rows -> gbuf (one copy, or one per row)
-    const int j0 = c * kChunk, n = min(kChunk, n_rows - j0);
+    int j0, n;
+    cm.rows(c, j0, n);
     mbar_arrive_expect_tx(&s_bar, (uint32_t)n * row_bytes);
     if (!cand) {
       bulk_load(gbuf, Wpre + (size_t)j0 * rowlen, (uint32_t)n * row_bytes, &s_bar);
@@ -246,12 +294,10 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     s_abort = 0;
     mbar_init(&s_bar, 1);
     fence_mbar_init();
-    const int c0 = tk.resolve(g, tk.draw(g));
+    const int c0 = (int)blockIdx.x < cm.n_chunks ? (int)blockIdx.x : -1;
     s_next[0] = c0;
-    if (c0 >= 0) {
-      issue_gate(c0);
-      t_pending = tk.draw(g);
-    }
+    if (c0 >= 0) issue_gate(c0);
+    t_pending = tk.draw(g);
   }
   stage_tokens<WT, NB>(xs, reinterpret_cast<const WT*>(p.x), B, d);
   __syncthreads();
@@ -357,13 +403,15 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
 
     // 1. gate and threshold for position j (neuron r; one per warp) from the prefetched rows
     mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
-    const int j = chunk * kChunk + warp;
-    const int r = j < n_rows ? neuron(j) : 0;
+    int j0, n_in;
+    cm.rows(chunk, j0, n_in);
+    const int j = j0 + warp;
+    const int r = warp < n_in ? neuron(j) : 0;
     float a[NB];
     bool any = false;
 #pragma unroll
     for (int b = 0; b < NB; ++b) a[b] = 0.f;
-    if (j < n_rows) {
+    if (warp < n_in) {
       float z[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) z[b] = 0.f;
@@ -429,9 +477,13 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     chunk = next;
   }
 
-  // ---------------------------------------------------------------- partials, then a grid count
+  // ---------------------------------------------------------------- partial sums, then one grid meeting
+  // The CTA adds its register partial of out into accumulator blockIdx % kFusedAccCopies with
+  // vector reductions in L2, issued the moment its chunks are done, so they overlap the other
+  // CTAs' last chunks; spreading the CTAs over several accumulators shortens the queue of
+  // reductions on each address.
   {
-    float* part = p.partial + (size_t)blockIdx.x * B * d;
+    float* accp = p.facc + (size_t)(blockIdx.x % kFusedAccCopies) * B * d;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       if (b < B) {
@@ -439,10 +491,10 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
         for (int k = 0; k < KD; ++k) {
           const int c = lane + k * kWarp;
           if (c < cpw) {
-            float4* dst = reinterpret_cast<float4*>(part + (size_t)b * d + (size_t)(warp * cpw + c) * EPV);
+            float* dst = accp + (size_t)b * d + (size_t)(warp * cpw + c) * EPV;
 #pragma unroll
             for (int e = 0; e < EPV; e += 4)
-              __stcg(dst + e / 4, make_float4(acc[b][k][e], acc[b][k][e + 1], acc[b][k][e + 2], acc[b][k][e + 3]));
+              red_add_v4(dst + e, acc[b][k][e], acc[b][k][e + 1], acc[b][k][e + 2], acc[b][k][e + 3]);
           }
         }
       }
@@ -451,93 +503,96 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    atomicAdd(&p.ctl[kCtlDone], 1u);
-    wait_at_least(&p.ctl[kCtlDone], gridDim.x, p.err);
+    // The arrival counter wraps back to zero on the last arrival (atomicInc); the others wait for
+    // that zero (their own arrival keeps it above zero until then), so it is ready for the next
+    // launch without a reset.  Every CTA has drawn its last ticket (and passed the predictor's
+    // count) before it arrives, so the last one also clears those counters for the next launch.
+    if (atomicInc(&p.ctl[kCtlDone], gridDim.x - 1u) == gridDim.x - 1u) {
+      for (int i = 0; i < kCounters; ++i) {
+        p.tickets[i * kCounterStride] = 0u;
+        p.tickets[i * kCounterStride + 1] = 0u;
+      }
+      p.ctl[kCtlY] = 0u;
+      __threadfence();  // with the counter read above: the other CTAs' sums are visible here
+    } else {
+      wait_zero(&p.ctl[kCtlDone], p.err);
+    }
   }
   __syncthreads();
 
   if (warp < kHalf / kWarp) {
-    // ------------------------------------------------------------ cross-CTA sum of the partials
-    // Slice s = columns [16 s, 16 s + 16).  Thread (grp, q) adds float4 q of the partials of CTAs
-    // grp, grp + 32, ... (all loads issued together); the 8 groups of a warp are folded with
-    // shuffles, the 4 warps in shared memory.
-    const int q = tid & 3, grp = tid >> 2;
-    const int n_slices = d / kSumCols;
-    for (int s = blockIdx.x; s < n_slices; s += gridDim.x) {
-      for (int b = 0; b < B; ++b) {
-        // every load is issued (rows past the grid read row 0 and are weighted 0), then summed
-        float4 x4[kSumLoads];
+    // ------------------------------------------------------------ out = the accumulators' sum
+    // CTA k takes an equal share of the B*d/4 float4 columns, writes their sum (plus the old out
+    // when accumulating) and clears them for the next launch.
+    const int n4 = B * d / 4;
+    const int i0 = (int)((long long)n4 * blockIdx.x / gridDim.x);
+    const int i1 = (int)((long long)n4 * (blockIdx.x + 1) / gridDim.x);
+    for (int i = i0 + tid; i < i1; i += kHalf) {
+      float4 s4[kFusedAccCopies];
 #pragma unroll
-        for (int i = 0; i < kSumLoads; ++i) {
-          const int c = grp + i * kSumRowsPar;
-          const int cc = c < (int)gridDim.x ? c : 0;
-          x4[i] = __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)cc * B + b) * d + (size_t)s * kSumCols) + q);
-        }
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < kFusedAccCopies; ++c)
+        s4[c] = __ldcg(reinterpret_cast<const float4*>(p.facc + (size_t)c * B * d) + i);
+      float4 t4 = s4[0];
 #pragma unroll
-        for (int i = 0; i < kSumLoads; ++i) {
-          const float wgt = grp + i * kSumRowsPar < (int)gridDim.x ? 1.f : 0.f;
-          sum.x = fmaf(wgt, x4[i].x, sum.x);
-          sum.y = fmaf(wgt, x4[i].y, sum.y);
-          sum.z = fmaf(wgt, x4[i].z, sum.z);
-          sum.w = fmaf(wgt, x4[i].w, sum.w);
-        }
-#pragma unroll
-        for (int o = 4; o < kWarp; o <<= 1) {
-          sum.x += __shfl_xor_sync(0xffffffffu, sum.x, o);
-          sum.y += __shfl_xor_sync(0xffffffffu, sum.y, o);
-          sum.z += __shfl_xor_sync(0xffffffffu, sum.z, o);
-          sum.w += __shfl_xor_sync(0xffffffffu, sum.w, o);
-        }
-        if (lane < 4) s_sum[warp][lane] = sum;
-        named_sync(1, kHalf);
-        if (tid < 4) {
-          float4 t4 = s_sum[0][tid];
-#pragma unroll
-          for (int w = 1; w < kHalf / kWarp; ++w) {
-            const float4 o4 = s_sum[w][tid];
-            t4.x += o4.x;
-            t4.y += o4.y;
-            t4.z += o4.z;
-            t4.w += o4.w;
-          }
-          const size_t o = (size_t)b * d + (size_t)s * kSumCols + tid * 4;
-          if (p.out_mode == CSFFN_OUT_BF16) {
-            bf16* ob = reinterpret_cast<bf16*>(p.out) + o;
-            ob[0] = __float2bfloat16_rn(t4.x);
-            ob[1] = __float2bfloat16_rn(t4.y);
-            ob[2] = __float2bfloat16_rn(t4.z);
-            ob[3] = __float2bfloat16_rn(t4.w);
-          } else {
-            float4* of = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o);
-            if (p.out_mode == CSFFN_OUT_F32_ACCUMULATE) {
-              const float4 prev = *of;
-              t4.x += prev.x;
-              t4.y += prev.y;
-              t4.z += prev.z;
-              t4.w += prev.w;
-            }
-            *of = t4;
-          }
-        }
-        named_sync(1, kHalf);
+      for (int c = 1; c < kFusedAccCopies; ++c) {
+        t4.x += s4[c].x;
+        t4.y += s4[c].y;
+        t4.z += s4[c].z;
+        t4.w += s4[c].w;
       }
+      if (p.out_mode == CSFFN_OUT_BF16) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(t4.x, t4.y), hi = __floats2bfloat162_rn(t4.z, t4.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(p.out)[i] = pk;
+      } else {
+        float4* of = reinterpret_cast<float4*>(p.out) + i;
+        if (p.out_mode == CSFFN_OUT_F32_ACCUMULATE) {
+          const float4 prev = *of;
+          t4.x += prev.x;
+          t4.y += prev.y;
+          t4.z += prev.z;
+          t4.w += prev.w;
+        }
+        *of = t4;
+      }
+#pragma unroll
+      for (int c = 0; c < kFusedAccCopies; ++c)
+        __stcg(reinterpret_cast<float4*>(p.facc + (size_t)c * B * d) + i, make_float4(0.f, 0.f, 0.f, 0.f));
     }
   } else {
     // ------------------------------------------------------------ compaction of the active list
     // CTA k owns the 32-position words [wa, wb); the kept positions before wa are counted from the
     // flag bytes (each 0 or 1, so the popcount of a 32-bit word of flags counts its kept rows).
-    // Position j is written out as its neuron (ascending, as the candidate list is).
+    // Position j is written out as its neuron (ascending, as the candidate list is).  The flags and
+    // activations of the first pass are loaded before that count, so the two round trips overlap.
     const int ct = tid - kHalf, cw = warp - kHalf / kWarp;
     const int n_words = (n_rows + kWarp - 1) / kWarp;
     const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
     const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
     if (wa < wb || blockIdx.x == gridDim.x - 1) {
+      bool f;
+      int nr;
+      float av[NB];
+      auto load_pass = [&](int w0) {  // flag, neuron and activations of position (w0 + cw) * 32 + lane
+        const int jp = (w0 + cw) * kWarp + lane;
+        const bool in = w0 + cw < wb && jp < n_rows;
+        f = in && __ldcg(p.flags + jp) != 0;
+        nr = in ? neuron(jp) : 0;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
+      };
+      load_pass(wa);
       uint32_t before = 0;
       const uint4* f4 = reinterpret_cast<const uint4*>(p.flags);
-      for (int i = ct; i < wa * 2; i += kHalf) {
-        const uint4 f = __ldcg(f4 + i);
-        before += __popc(f.x) + __popc(f.y) + __popc(f.z) + __popc(f.w);
+      for (int i0 = ct; i0 < wa * 2; i0 += kHalf * kCountLoads) {  // each batch's loads issued together
+        uint4 fw[kCountLoads];
+#pragma unroll
+        for (int u = 0; u < kCountLoads; ++u)
+          fw[u] = i0 + u * kHalf < wa * 2 ? __ldcg(f4 + i0 + u * kHalf) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < kCountLoads; ++u) before += __popc(fw[u].x) + __popc(fw[u].y) + __popc(fw[u].z) + __popc(fw[u].w);
       }
       before = warp_sum_u32(before);
       if (lane == 0) s_cnt[cw] = before;
@@ -547,13 +602,6 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       for (int w = 0; w < kHalf / kWarp; ++w) base += s_cnt[w];
       named_sync(2, kHalf);
       for (int w0 = wa; w0 < wb; w0 += kHalf / kWarp) {
-        const int w = w0 + cw;
-        const int jp = w * kWarp + lane;
-        const bool in = w < wb && jp < n_rows;
-        const bool f = in && __ldcg(p.flags + jp) != 0;
-        float av[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
         const uint32_t m = __ballot_sync(0xffffffffu, f);
         if (lane == 0) s_cnt[cw] = __popc(m);
         named_sync(2, kHalf);
@@ -565,31 +613,16 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
         }
         if (f) {
           const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
-          p.idx[pos] = neuron(jp);
+          p.idx[pos] = nr;
 #pragma unroll
           for (int b = 0; b < NB; ++b)
             if (b < B) p.a_val[(size_t)b * h + pos] = av[b];
         }
         base = total;
         named_sync(2, kHalf);
+        load_pass(w0 + kHalf / kWarp);
       }
       if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
-    }
-  }
-
-  // ---------------------------------------------------------------- the last CTA out resets
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(&p.ctl[kCtlExit], 1u) == gridDim.x - 1) {
-      for (int i = 0; i < kCounters; ++i) {
-        p.tickets[i * kCounterStride] = 0u;
-        p.tickets[i * kCounterStride + 1] = 0u;
-      }
-      p.ctl[kCtlDone] = 0u;
-      p.ctl[kCtlY] = 0u;
-      p.ctl[kCtlExit] = 0u;
-      __threadfence();
     }
   }
 }
@@ -604,7 +637,7 @@ static size_t fused_smem_bytes(int d, int nb, size_t es, int rank = 0) {
 // Down-slice width per lane (16-byte columns) for a shape, 0 when the fused kernel does not take it.
 static int fused_kd(int d, int B, int wdtype) {
   const int epv = wdtype == CSFFN_F32 ? 4 : 8;
-  if (d % (epv * kFusedWarps) != 0 || d % kSumCols != 0) return 0;
+  if (d % (epv * kFusedWarps) != 0) return 0;
   const int cpw = d / epv / kFusedWarps;
   const int kd = cpw <= 32 ? 1 : cpw <= 64 ? 2 : cpw <= 128 ? 4 : 0;
   // register budget: the down accumulators (tokens x kd x epv floats) beside a streamed row
@@ -625,9 +658,7 @@ static cudaError_t fused_t(FusedArgs a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   if (occ > 2) occ = 2;
-  int grid = sm_count() * occ;
-  if (grid > a.partial_rows / a.B) grid = a.partial_rows / a.B;
-  if (grid < 1) return cudaErrorInvalidConfiguration;
+  const int grid = sm_count() * occ;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kFusedThreads);

@@ -40,6 +40,7 @@ struct WsLayout {
   size_t err;        // uint32 error word (+ pad)
   size_t slice_ctr;  // uint32 [kSliceUsers][kMaxSlices]
   size_t tickets;    // uint32 [64][32]                 chunk-ticket counters, 128 B apart (fused path)
+  size_t facc;       // fp32 [kFusedAccCopies][kFusedMaxBatch][CSFFN_MAX_D] out accumulators (fused path)
   size_t status;     // uint64 [kNumCtl][max_chunks]   look-back status words
   size_t control_end;
   size_t vbuf;       // fp32 [max_batch][h]            v = a * u (sparse) or act(z)*u (dense)
@@ -54,15 +55,11 @@ struct WsLayout {
 };
 
 constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
-constexpr int kFusedMaxCtas = 320;  // CTAs of the fused step (2 per SM) with a partial each
 constexpr int kFusedMaxBatch = 4;
+constexpr int kFusedAccCopies = 4;  // fused step: CTA k adds into accumulator k % kFusedAccCopies
 
-// Rows of d floats in the partial region.
-__host__ __device__ inline int partial_rows(int max_batch) {
-  const int ranges = kMaxRowRanges * max_batch;
-  const int fused = kFusedMaxCtas * (max_batch < kFusedMaxBatch ? max_batch : kFusedMaxBatch);
-  return ranges > fused ? ranges : fused;
-}
+// Rows of d floats in the partial region (one per row range of the sparse/dense forward).
+__host__ __device__ inline int partial_rows(int max_batch) { return kMaxRowRanges * max_batch; }
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -75,6 +72,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   o = align_up(o, 128);
   L.tickets = o;    o += sizeof(uint32_t) * 64 * 32;
   o = align_up(o, 256);
+  L.facc = o;       o += sizeof(float) * (size_t)kFusedAccCopies * kFusedMaxBatch * CSFFN_MAX_D;
+  o = align_up(o, 256);
   L.max_chunks = (h + kChunkRows - 1) / kChunkRows;
   L.status = o;     o += sizeof(uint64_t) * (size_t)kNumCtl * L.max_chunks;
   o = align_up(o, 256);
@@ -85,7 +84,7 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   o = align_up(o, 256);
   L.flags = o;      o += align_up((size_t)h, 16);
   o = align_up(o, 256);
-  // partials: one per row range of the sparse/dense forward, or one per CTA of the fused step
+  // partials: one per row range of the sparse/dense forward
   L.partial = o;    o += sizeof(float) * (size_t)partial_rows(max_batch) * d;
   o = align_up(o, 256);
   L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);

@@ -127,10 +127,8 @@ struct FusedArgs {
   float* ybuf;                // [B, rank] scratch: y = x U_r
   float* afull;      // [B, h] scratch: kept activation per row position
   uint8_t* flags;    // [h] scratch: keep flag per row position (16-byte aligned)
-  float* partial;    // [partial_rows / B][B, d] scratch: one fp32 partial of out per CTA
-  int partial_rows;  // capacity of partial in rows of d floats
-  int chunk_rows;    // neuron rows per chunk (set by the launcher)
-  uint32_t* ctl;     // fused control words (done and exit counters), zero between launches
+  float* facc;      // fp32 [kFusedAccCopies][B, d] accumulators of out, zero between launches
+  uint32_t* ctl;     // fused control words (arrival counter, generation), zero before first use
   uint32_t* tickets; // [32 * 32] chunk-ticket counters and dry flags, 128 bytes apart
   uint32_t* err;
   int32_t* idx;

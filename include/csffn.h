@@ -108,8 +108,9 @@ const char* csffn_status_string(int status);
  * Returns 0 if the arguments are invalid. */
 size_t csffn_workspace_size(const csffn_layer* layer, int max_batch, int max_rank);
 
-/* Zero the workspace's control words; required once before first use and after
- * a CSFFN_ERR_TIMEOUT.  Asynchronous on `stream`. */
+/* Zero the workspace's control region (counters, the one-launch step's output
+ * accumulators); required once before first use and after a CSFFN_ERR_TIMEOUT.
+ * Asynchronous on `stream`. */
 csffn_status csffn_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the device-side error word of `ws`.
@@ -147,13 +148,15 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
  * csffn_sparse_ffn_forward computes, with the same outputs (idx, *count, a_val as gate_mask;
  * out as sparse_ffn_forward).  [CATS] abstract: the gate GEMV, the compare and the flag-gated
  * GEMV of one FFN layer.  One pass over dynamically assigned chunks of neuron rows runs the gate,
- * the threshold, and the up and down projections of the kept rows; after a grid-wide count
- * (cooperative launch) the per-CTA partial outputs are summed and idx / a_val / count compacted.
+ * the threshold, and the up and down projections of the kept rows.  Each CTA adds its partial
+ * output into fp32 accumulators in the workspace as soon as its rows are done; after a grid-wide
+ * count (cooperative launch) the accumulators become out and are cleared for the next call, and
+ * idx / a_val / count are compacted.
  * One launch pays one ramp-up and one tail instead of three.  Runs for 1 <= B <= 4 when
  * d % 128 == 0 (bf16; d % 64 for fp32) and the tokens fit in shared memory beside the weight
  * buffers; other shapes fall back to the two-call path inside this call.  The mask and a_val are
  * bit-for-bit repeatable; out may differ from launch to launch in the last bits (rows reach CTAs
- * dynamically, so the order of the final fp32 sum varies).  cand_idx / cand_count (both or
+ * dynamically and the CTAs' fp32 partial sums are added in arrival order).  cand_idx / cand_count (both or
  * neither): as in csffn_gate_mask, only the listed neurons (ascending, device count) are
  * considered, e.g. the set csffn_predict_lowrank predicts ([SVDP] Fig. 3: the gate runs on the
  * predicted set; with act = RELU and t = 0 the kept set is {z > 0} within it).  ws sized by
