@@ -128,27 +128,35 @@ template <int NB, int KD> struct FusedDownRows {
   static constexpr int value = NB * KD <= 2 ? 8 : (NB * KD <= 4 ? 4 : 2);  // a whole chunk at batch 1
 };
 
-// Chunks in row order: kChunk rows each, then (for the last kTailGrids grid widths of chunks)
-// kTailChunk rows each, so the work a CTA still holds when the tickets run out is small and the
-// CTAs finish close together.
+// Chunks in row order: `big` rows each, then `small` rows each for the last `tail` rows (at
+// least), so that the work a CTA still holds when the tickets run out is small and the CTAs
+// finish close together.
 struct ChunkMap {
-  int n_rows, n_big, n_chunks;
-  __device__ void init(int rows, int grid) {
+  int n_rows, big, small, n_big, n_chunks;
+  __device__ void init(int rows, int big_rows, int small_rows, int tail) {
     n_rows = rows;
-    const int tail = kTailGrids * grid * kTailChunk;  // rows wanted in small chunks
-    n_big = rows > tail ? (rows - tail) / kChunk : 0;
-    n_chunks = n_big + (rows - n_big * kChunk + kTailChunk - 1) / kTailChunk;
+    big = big_rows;
+    small = small_rows;
+    n_big = rows > tail ? (rows - tail) / big : 0;
+    n_chunks = n_big + (rows - n_big * big + small - 1) / small;
   }
   __device__ void rows(int c, int& j0, int& n) const {
     if (c < n_big) {
-      j0 = c * kChunk;
-      n = kChunk;
+      j0 = c * big;
+      n = big;
     } else {
-      j0 = n_big * kChunk + (c - n_big) * kTailChunk;
-      n = min(kTailChunk, n_rows - j0);
+      j0 = n_big * big + (c - n_big) * small;
+      n = min(small, n_rows - j0);
     }
   }
 };
+
+// Predictor mode: at most this many groups of kChunk V_r rows per chunk (and 64 KB of rows).
+constexpr int kPredSubMax = 16;
+__host__ __device__ inline int pred_sub_max(int rank, int es) {
+  const int r = 65536 / (kChunk * rank * es);
+  return r < 1 ? 1 : (r > kPredSubMax ? kPredSubMax : r);
+}
 
 // Tickets, drawn by thread 0, for the chunks after the first grid width (CTA b starts on chunk b
 // without a draw).  Counter g hands out chunks base + [lo(g), lo(g + 1)); a counter found dry is
@@ -241,7 +249,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   __shared__ int s_abort;
   __shared__ float s_v[kQueueBatch][NB];        // v of the batch being flushed
   __shared__ int s_drow[kQueueBatch];            // its neurons
-  __shared__ uint8_t s_keep[2][kChunk];          // keep flags of the chunk (by parity)
+  __shared__ uint8_t s_keep[2][kChunk];          // keep flags of the chunk or round (by parity)
+  __shared__ int s_plist[PRED ? 2 : 1][kFusedWarps][kPredSubMax];  // predictor: predicted rows per warp
+  __shared__ int s_pcnt[PRED ? 2 : 1][kFusedWarps];
   __shared__ int s_qrow[kQueueSlots];            // queued kept rows: neuron
   __shared__ float s_qa[kQueueSlots][NB];        // and kept activations per token
   __shared__ int s_next[2];
@@ -251,8 +261,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   const int cpw = d / EPV / kFusedWarps;  // 16-byte columns of W_down^T owned by each warp
   WT* xs = reinterpret_cast<WT*>(smem_raw);
   const int rowlen = PRED ? p.rank : d;  // elements of a prefetched row (V_r or W_gate)
-  WT* gbuf = xs + (size_t)NB * d;         // prefetched rows of the current chunk [kChunk][rowlen]
-  float* ys = reinterpret_cast<float*>(gbuf + (size_t)kChunk * rowlen);  // predictor mode: y [NB][rank]
+  WT* gbuf = xs + (size_t)NB * d;         // prefetched rows of the current chunk [chunk rows][rowlen]
+  // predictor mode: y [NB][rank] after the largest chunk of V_r rows
+  float* ys = reinterpret_cast<float*>(gbuf + (size_t)kChunk * (PRED ? pred_sub_max(p.rank, (int)sizeof(WT)) : 1) * rowlen);
   const WT* Wg = reinterpret_cast<const WT*>(p.W_gate);
   const WT* Wu = reinterpret_cast<const WT*>(p.W_up);
   const WT* Wd = reinterpret_cast<const WT*>(p.W_down_t);
@@ -266,7 +277,15 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   auto neuron = [&](int j) { return cand ? __ldg(cand + j) : j; };
 
   ChunkMap cm;
-  cm.init(n_rows, (int)gridDim.x);
+  if constexpr (PRED) {
+    // one chunk per CTA where the rows allow: the work per row is a few hundred bytes of V_r, so a
+    // chunk's round trips, not its bytes, set its time
+    const int per = (n_rows + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int cs = max(kChunk, min((per + kChunk - 1) / kChunk * kChunk, kChunk * pred_sub_max(p.rank, (int)sizeof(WT))));
+    cm.init(n_rows, cs, cs, 0);
+  } else {
+    cm.init(n_rows, kChunk, kTailChunk, kTailGrids * (int)gridDim.x * kTailChunk);
+  }
   Tickets tk;
   tk.ctr = p.tickets;
   tk.base = min((int)gridDim.x, cm.n_chunks);
@@ -397,73 +416,47 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
     q_head += n;
   };
 
-  int chunk = s_next[0];
-  for (int it = 0; chunk >= 0; ++it) {
-    const int buf = it & 1;
-
-    // 1. gate and threshold for position j (neuron r; one per warp) from the prefetched rows
-    mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
-    int j0, n_in;
-    cm.rows(chunk, j0, n_in);
-    const int j = j0 + warp;
-    const int r = warp < n_in ? neuron(j) : 0;
-    float a[NB];
+  // Threshold one gate row: per token the activation of z + beta against t; records the keep flag
+  // and the kept activations of position j and returns whether any token keeps the row.
+  auto decide = [&](int j, float (&z)[NB], float beta, float (&a)[NB]) {
     bool any = false;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) a[b] = 0.f;
-    if (warp < n_in) {
-      float z[NB];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) z[b] = 0.f;
-      const float beta = p.bias ? __ldg(p.bias + r) : 0.f;
-      bool gate_row = true;
-      if constexpr (PRED) {
-        // predictor: p = y . V_r[r] + beta against tau_r (union over tokens); the gate row streams
-        // from HBM only for a predicted neuron
-        smem_dot_f32<WT, NB>(gbuf + (size_t)warp * rowlen, ys, rowlen, lane, z);
-        const float tau = __ldg(p.tau + r);
-        bool pred = false;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          pred |= b < B && warp_sum(z[b]) + beta > tau;
-          z[b] = 0.f;
-        }
-        gate_row = pred;
-        if (pred) row_dot<WT, NB, FusedGateU<NB>::value>(Wg + (size_t)r * d, xs, d, lane, z);
-      } else {
-        smem_row_dot<WT, NB>(gbuf + (size_t)warp * d, xs, d, lane, z);
-      }
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float ab = gate_act(warp_sum(z[b]) + beta, p.act);
-        const bool kb = gate_row && b < B && fabsf(ab) > p.t;
-        a[b] = kb ? ab : 0.f;
-        any |= kb;
-      }
-      if (lane == 0) {
-        p.flags[j] = any ? 1 : 0;
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-          if (b < B) p.afull[(size_t)b * h + j] = a[b];
-      }
+    for (int b = 0; b < NB; ++b) {
+      const float ab = gate_act(warp_sum(z[b]) + beta, p.act);
+      const bool kb = b < B && fabsf(ab) > p.t;
+      a[b] = kb ? ab : 0.f;
+      any |= kb;
     }
-    if (lane == 0) s_keep[buf][warp] = any ? 1 : 0;
+    if (lane == 0) {
+      p.flags[j] = any ? 1 : 0;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (b < B) p.afull[(size_t)b * h + j] = a[b];
+    }
+    return any;
+  };
+  // Thread 0 resolves the ticket drawn a chunk ago and publishes it; after the block barrier (the
+  // step's shared writes are visible, gbuf is free) it issues that chunk's copy and draws again.
+  auto advance = [&](int buf) {
     int cn = -1;
     if (tid == 0) {
-      cn = tk.resolve(g, t_pending);  // drawn a chunk ago: its round trip is over
+      cn = tk.resolve(g, t_pending);
       s_next[buf ^ 1] = cn;
     }
-    __syncthreads();  // keep flags and the next chunk are visible; gbuf is free
+    __syncthreads();
     if (tid == 0 && cn >= 0) {
       fence_proxy_async_smem();
-      issue_gate(cn);  // prefetch the next chunk's rows
+      issue_gate(cn);
       t_pending = tk.draw(g);
     }
-
-    // 2. queue the chunk's kept rows; up and down run on batches of kQueueBatch queued rows
+    return s_next[buf ^ 1];
+  };
+  // Append the kept rows of one step (warp w's row r when keep[w]) to the queue, in warp order, and
+  // flush a batch once kQueueBatch are waiting.
+  auto enqueue = [&](bool any, int r, const float (&a)[NB], const uint8_t* keep) {
     uint32_t mask = 0;
 #pragma unroll
-    for (int jj = 0; jj < kChunk; ++jj) mask |= s_keep[buf][jj] ? 1u << jj : 0u;
+    for (int jj = 0; jj < kChunk; ++jj) mask |= keep[jj] ? 1u << jj : 0u;
     if (any && lane == 0) {
       const int slot = (q_tail + __popc(mask & ((1u << warp) - 1u))) & (kQueueSlots - 1);
       s_qrow[slot] = r;
@@ -471,8 +464,105 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       for (int b = 0; b < NB; ++b) s_qa[slot][b] = a[b];
     }
     q_tail += __popc(mask);
-    const int next = s_next[buf ^ 1];
     if (q_tail - q_head >= kQueueBatch) flush(kQueueBatch);
+  };
+
+  int chunk = s_next[0];
+  int kr = 0;  // predictor mode: rounds so far (parity of their keep flags)
+  for (int it = 0; chunk >= 0; ++it) {
+    const int buf = it & 1;
+    mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
+    int j0, n_in;
+    cm.rows(chunk, j0, n_in);
+    int next;
+    if constexpr (!PRED) {
+      // 1. gate and threshold for position j (neuron r; one per warp) from the prefetched rows
+      const int j = j0 + warp;
+      const int r = warp < n_in ? neuron(j) : 0;
+      float a[NB];
+      bool any = false;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) a[b] = 0.f;
+      if (warp < n_in) {
+        float z[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) z[b] = 0.f;
+        const float beta = p.bias ? __ldg(p.bias + r) : 0.f;
+        smem_row_dot<WT, NB>(gbuf + (size_t)warp * d, xs, d, lane, z);
+        any = decide(j, z, beta, a);
+      }
+      if (lane == 0) s_keep[buf][warp] = any ? 1 : 0;
+      next = advance(buf);
+      // 2. queue the chunk's kept rows; up and down run on batches of kQueueBatch queued rows
+      enqueue(any, r, a, s_keep[buf]);
+    } else {
+      // a. the prediction p = y . V_r[j] + beta_j against tau_j (union over tokens) for every row of
+      //    the chunk, warp w taking rows w, w + 8, ...; a row not predicted is final here.  Lane i
+      //    fetches tau and beta of the warp's row i, so those loads overlap.
+      float tau_l = 0.f, beta_l = 0.f;
+      {
+        const int qi = warp + lane * kFusedWarps;
+        if (lane < kPredSubMax && qi < n_in) {
+          tau_l = __ldg(p.tau + neuron(j0 + qi));
+          beta_l = p.bias ? __ldg(p.bias + neuron(j0 + qi)) : 0.f;
+        }
+      }
+      int pc = 0;
+      for (int i = 0; warp + i * kFusedWarps < n_in; ++i) {
+        const int q = warp + i * kFusedWarps;
+        float z[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) z[b] = 0.f;
+        smem_dot_f32<WT, NB>(gbuf + (size_t)q * rowlen, ys, rowlen, lane, z);
+        const float tau = __shfl_sync(0xffffffffu, tau_l, i), beta = __shfl_sync(0xffffffffu, beta_l, i);
+        bool pred = false;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) pred |= b < B && warp_sum(z[b]) + beta > tau;
+        if (pred) {
+          if (lane == 0) s_plist[buf][warp][pc] = q;
+          ++pc;
+        } else if (lane == 0) {
+          p.flags[j0 + q] = 0;
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            if (b < B) p.afull[(size_t)b * h + j0 + q] = 0.f;
+        }
+      }
+      if (lane == 0) s_pcnt[buf][warp] = pc;
+      next = advance(buf);
+      // b. rounds of up to kFusedWarps predicted rows: warp w streams the W_gate row of one from HBM
+      //    and thresholds it; each round's kept rows go to the queue
+      int pre[kFusedWarps + 1];
+      pre[0] = 0;
+#pragma unroll
+      for (int w = 0; w < kFusedWarps; ++w) pre[w + 1] = pre[w] + s_pcnt[buf][w];
+      const int P = pre[kFusedWarps];
+      for (int base = 0; base < P; base += kFusedWarps) {
+        const int k = base + warp;
+        int r = 0;
+        float a[NB];
+        bool any = false;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) a[b] = 0.f;
+        if (k < P) {
+          int w = 0;
+#pragma unroll
+          for (int ww = 1; ww < kFusedWarps; ++ww) w += k >= pre[ww] ? 1 : 0;
+          const int jq = j0 + s_plist[buf][w][k - pre[w]];
+          r = neuron(jq);
+          const float beta = p.bias ? __ldg(p.bias + r) : 0.f;
+          float z[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) z[b] = 0.f;
+          row_dot<WT, NB, FusedGateU<NB>::value>(Wg + (size_t)r * d, xs, d, lane, z);
+          any = decide(jq, z, beta, a);
+        }
+        if (lane == 0) s_keep[kr & 1][warp] = any ? 1 : 0;
+        __syncthreads();  // the round's keep flags are visible
+        enqueue(any, r, a, s_keep[kr & 1]);
+        ++kr;
+      }
+    }
     if (next < 0 && q_tail > q_head) flush(q_tail - q_head);  // this CTA's last chunk: drain
     chunk = next;
   }
@@ -630,7 +720,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
 // Dynamic shared memory: the staged tokens and one chunk of prefetched rows (W_gate, or V_r in
 // predictor mode, with the predictor's y beside them).
 static size_t fused_smem_bytes(int d, int nb, size_t es, int rank = 0) {
-  if (rank > 0) return (size_t)nb * d * es + (size_t)kChunk * rank * es + (size_t)nb * rank * sizeof(float);
+  if (rank > 0)
+    return (size_t)nb * d * es + (size_t)kChunk * pred_sub_max(rank, (int)es) * rank * es +
+           (size_t)nb * rank * sizeof(float);
   return (size_t)(nb + kChunk) * d * es;
 }
 
