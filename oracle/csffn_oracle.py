@@ -6,7 +6,8 @@ this module: only the tests, ``__graft_entry__.smoke()`` and the
 no code with the CUDA library.
 
 Every function computes the plain definition in float64 with numpy (matrix
-products are the only library primitive used), on exactly the operand bits
+products, the SVD, a Cholesky factorisation and a linear solve are the only
+library primitives used), on exactly the operand bits
 the GPU receives (bf16 bit patterns as uint16, or float32).  No blocking,
 fusion or reordering: the sparse method reaches the same result faster.
 
@@ -30,7 +31,9 @@ notes): the CATS threshold applies to the gate output SiLU(z) with strict
 ``|a| > t``; the quantile is the lower order statistic v_(ceil(s*M)) without
 interpolation; t is one scalar per layer pooled over neurons x calibration
 vectors; the SVD predictor factors W_gate^T = U S V^T as U_r = U[:, :r] S_r
-(stored transposed, [r, d]) and V_r = V[:, :r] ([h, r]); tau_i is the
+(stored transposed, [r, d]) and V_r = V[:, :r] ([h, r]), and its data-whitened
+variant takes the truncated SVD of L^T W_gate^T with C = X^T X = L L^T over the
+calibration rows (plus a small ridge); tau_i is the
 per-neuron lower order statistic of the predictor output at q; the gate bias
 is an explicit additive vector; RMSNorm has unit gain and eps = 1e-6.
 """
@@ -179,6 +182,31 @@ def svd_factors(w_gate, r: int) -> tuple:
     """
     u, s, vt = np.linalg.svd(decode(w_gate).T, full_matrices=False)
     return (u[:, :r] * s[None, :r]).T.copy(), vt[:r, :].T.copy()
+
+
+WHITEN_RIDGE = 1e-6
+
+
+def svd_factors_whitened(w_gate, r: int, x_cal, ridge: float = WHITEN_RIDGE) -> tuple:
+    """[SVDP] abstract ("truncation-aware" SVD) and Table 3 ("+ Data whitening"): the rank-r
+    factors of W_gate^T that best reproduce the gate pre-activations of the calibration inputs.
+
+    Reading (the pages name the step but print no formula): among rank-r d x h matrices M,
+    minimise ||X (W_gate^T - M)||_F over the calibration rows X [N, d].  With
+    C = X^T X + lambda I = L L^T (Cholesky; lambda = ridge * trace(X^T X) / d keeps C
+    definite when N < d), ||X A||_F^2 = ||L^T A||_F^2 up to the ridge, so the optimum is the
+    truncated SVD of the whitened matrix, L^T W_gate^T = U S V^T, mapped back:
+    M = L^{-T} U_r S_r V_r^T.  Returns (U_r^T [r, d] = (L^{-T} U[:, :r] S_r)^T, V_r [h, r]) in
+    float64, the same layout as svd_factors; the predictor is unchanged (p = x U_r V_r^T + beta).
+    """
+    xs = _tokens(x_cal)
+    c = xs.T @ xs
+    d = c.shape[0]
+    c = c + (ridge * np.trace(c) / d) * np.eye(d)
+    low = np.linalg.cholesky(c)  # C = L L^T, L lower triangular
+    u, s, vt = np.linalg.svd(low.T @ decode(w_gate).T, full_matrices=False)
+    u_r = np.linalg.solve(low.T, u[:, :r] * s[None, :r])  # L^{-T} U_r S_r
+    return u_r.T.copy(), vt[:r, :].T.copy()
 
 
 def predict(x, u_rt, v_r, bias=None) -> np.ndarray:

@@ -270,6 +270,58 @@ def test_svd_singular_values_and_truncation_error():
     assert err == pytest.approx(np.sqrt(np.sum(sv[r:] ** 2)), rel=1e-10)
 
 
+def _aniso_tokens(n, d, seed=7, spread=5.0):
+    """Rows g A with A = diag(spectrum) Q: a fixed input covariance with eigenvalues spread over a
+    factor spread^2, so that the data-whitened and the naive factors differ (float32 operands)."""
+    rng = np.random.default_rng(seed)
+    q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    spec = np.geomspace(1.0, 1.0 / spread, d)
+    return (rng.standard_normal((n, d)) @ (spec[:, None] * q)).astype(np.float32)
+
+
+def test_whitened_svd_is_the_best_rank_r_fit_on_calibration():
+    """With no ridge and N >= d, X (U_r V_r^T) is the truncated SVD of X W_gate^T itself (an
+    independent route: X = Q R with orthonormal Q, so the X-weighted optimum is the plain
+    Eckart-Young optimum of X W_gate^T), and its error beats the naive factors' on X."""
+    d, h, n, r = 24, 40, 200, 6
+    layer = _tiny_layer(d, h)
+    x = _aniso_tokens(n, d)
+    xd, w = _f64(x), _f64(layer.w_gate)
+    urt, vr = oracle.svd_factors_whitened(layer.w_gate, r, x, ridge=0.0)
+    assert urt.shape == (r, d) and vr.shape == (h, r)
+    fit = xd @ urt.T @ vr.T
+    u, s, vt = np.linalg.svd(xd @ w.T, full_matrices=False)
+    best = (u[:, :r] * s[None, :r]) @ vt[:r, :]
+    np.testing.assert_allclose(fit, best, atol=1e-10 * np.abs(best).max())
+    err_w = np.linalg.norm(xd @ w.T - fit)
+    assert err_w == pytest.approx(np.sqrt(np.sum(s[r:] ** 2)), rel=1e-10)
+    urt_n, vr_n = oracle.svd_factors(layer.w_gate, r)
+    err_n = np.linalg.norm(xd @ w.T - xd @ urt_n.T @ vr_n.T)
+    assert err_w < 0.9 * err_n
+    # the predictor reads them as it reads the naive factors
+    np.testing.assert_allclose(oracle.predict(x[:3], urt, vr), fit[:3], rtol=1e-12)
+
+
+def test_whitened_svd_full_rank_and_isotropic_data():
+    d, h = 20, 32
+    layer = _tiny_layer(d, h)
+    w = _f64(layer.w_gate)
+    x = _aniso_tokens(60, d)
+    urt, vr = oracle.svd_factors_whitened(layer.w_gate, d, x)
+    np.testing.assert_allclose(vr @ urt, w, atol=1e-10)  # full rank: exact whatever the data
+    # X^T X proportional to I (orthonormal columns, scaled): whitening changes nothing
+    q, _ = np.linalg.qr(np.random.default_rng(3).standard_normal((80, d)))
+    xi = 2.5 * q
+    for r in (3, 7):
+        urt_w, vr_w = oracle.svd_factors_whitened(layer.w_gate, r, xi)
+        urt_n, vr_n = oracle.svd_factors(layer.w_gate, r)
+        np.testing.assert_allclose(vr_w @ urt_w, vr_n @ urt_n, atol=1e-9)
+    # the ridge only matters where the calibration rows leave C singular (N < d)
+    urt_0, vr_0 = oracle.svd_factors_whitened(layer.w_gate, 5, x, ridge=0.0)
+    urt_1, vr_1 = oracle.svd_factors_whitened(layer.w_gate, 5, x)
+    np.testing.assert_allclose(vr_1 @ urt_1, vr_0 @ urt_0, atol=1e-4 * np.abs(w).max())
+
+
 # ----------------------------------------------------------------------------- invariants
 
 def test_reglu_t0_equals_dense():
@@ -337,6 +389,8 @@ PIN_TESTS = [
     lambda: test_per_neuron_calibration_matches_numpy(),
     lambda: test_svd_full_rank_reconstructs_gate(),
     lambda: test_svd_singular_values_and_truncation_error(),
+    lambda: test_whitened_svd_is_the_best_rank_r_fit_on_calibration(),
+    lambda: test_whitened_svd_full_rank_and_isotropic_data(),
     lambda: test_silu_matches_scipy_expit(),
 ]
 
@@ -368,6 +422,24 @@ def _mut_svd_no_sigma(w_gate, r):
     return u[:, :r].T.copy(), vt[:r, :].T.copy()
 
 
+def _mut_whiten_untransposed(w_gate, r, x_cal, ridge=oracle.WHITEN_RIDGE):
+    xs = oracle.decode(x_cal)
+    c = xs.T @ xs
+    c = c + (ridge * np.trace(c) / c.shape[0]) * np.eye(c.shape[0])
+    low = np.linalg.cholesky(c)
+    u, s, vt = np.linalg.svd(low @ oracle.decode(w_gate).T, full_matrices=False)
+    return np.linalg.solve(low, u[:, :r] * s[None, :r]).T.copy(), vt[:r, :].T.copy()
+
+
+def _mut_whiten_not_mapped_back(w_gate, r, x_cal, ridge=oracle.WHITEN_RIDGE):
+    xs = oracle.decode(x_cal)
+    c = xs.T @ xs
+    c = c + (ridge * np.trace(c) / c.shape[0]) * np.eye(c.shape[0])
+    low = np.linalg.cholesky(c)
+    u, s, vt = np.linalg.svd(low.T @ oracle.decode(w_gate).T, full_matrices=False)
+    return (u[:, :r] * s[None, :r]).T.copy(), vt[:r, :].T.copy()
+
+
 def _mut_up_uses_gate(x, layer):
     return oracle.csffn_oracle._tokens(x) @ oracle.decode(layer.w_gate).T
 
@@ -386,6 +458,8 @@ MUTANTS = {
     "mask_ge": ("cats_mask", _mut_mask_ge),
     "rank_floor": ("order_statistic_rank", _mut_rank_floor),
     "svd_no_sigma": ("svd_factors", _mut_svd_no_sigma),
+    "whiten_untransposed": ("svd_factors_whitened", _mut_whiten_untransposed),
+    "whiten_not_mapped_back": ("svd_factors_whitened", _mut_whiten_not_mapped_back),
     "up_uses_gate": ("up_projection", _mut_up_uses_gate),
     "reglu_ignores_pred": ("reglu_sequential", _mut_reglu_ignores_pred),
 }
