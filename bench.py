@@ -7,8 +7,9 @@ on 512 seeded calibration vectors at 50% target sparsity (70% and 90% and the de
 path of the same library are measured too and reported under "detail").
 
 A step is one CATS decode of one layer through csffn_cats_ffn_forward: gate GEMV + SiLU
-+ threshold + gathered up projection, a grid barrier, then the gathered down projection
-and the compaction of the active list, in one kernel launch.  The two-call path
++ threshold, the gathered up and down projections of the kept rows, then one grid meeting,
+the sum of the CTAs' partial outputs and the compaction of the active list, in one kernel
+launch.  The two-call path
 (csffn_gate_mask then csffn_sparse_ffn_forward, three kernels) is reported under "detail".  The
 timed steps rotate over 8 distinct layer weight sets (2.2 GB, many times the 126 MB L2)
 so no step reads weights that an earlier step left in L2.  K steps are captured in one
