@@ -203,6 +203,24 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
   return cuda_status(launch_down(dn, layer->wdtype, s));
 }
 
+namespace {
+
+// Every check of a CATS step with 1 <= B <= CSFFN_MAX_BATCH, whichever path runs it (the one-launch
+// kernel, or the gate mask then the gathered up/down), so that a rejected call launches nothing.
+csffn_status check_cats_step(const csffn_layer* layer, const void* x, int B, float t, const int32_t* idx,
+                             const float* a_val, const void* out, void* ws, size_t ws_bytes) {
+  if (!x || !idx || !a_val || !out || std::isnan(t)) return CSFFN_ERR_INVALID_ARG;
+  csffn_status st = check_weights(layer, true, true, true);
+  if (st != CSFFN_OK) return st;
+  if (!aligned16(x) || !aligned16(out)) return CSFFN_ERR_ALIGNMENT;
+  if (!cats_fused_supported(layer->d, B, layer->wdtype) &&
+      (size_t)batch_tier(B) * layer->d * esize(layer->wdtype) > kMaxDynSmem)
+    return CSFFN_ERR_UNSUPPORTED_SHAPE;
+  return check_ws(ws, ws_bytes, ws_layout(layer->d, layer->h, B, 0).ybuf);
+}
+
+}  // namespace
+
 csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
                                     const int32_t* cand_idx, const int32_t* cand_count,
                                     int32_t* idx, int32_t* count, float* a_val,
@@ -215,16 +233,13 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   if (!count) return CSFFN_ERR_INVALID_ARG;
   if ((cand_idx == nullptr) != (cand_count == nullptr)) return CSFFN_ERR_INVALID_ARG;
   if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
+  if ((st = check_cats_step(layer, x, B, t, idx, a_val, out, ws, ws_bytes)) != CSFFN_OK) return st;
   if (!cats_fused_supported(layer->d, B, layer->wdtype)) {
     st = csffn_gate_mask(layer, x, B, t, cand_idx, cand_count, idx, count, a_val, ws, ws_bytes, stream);
     if (st != CSFFN_OK) return st;
     return csffn_sparse_ffn_forward(layer, x, B, idx, count, a_val, out, out_mode, ws, ws_bytes, stream);
   }
-  if (!x || !idx || !a_val || !out || std::isnan(t)) return CSFFN_ERR_INVALID_ARG;
-  if ((st = check_weights(layer, true, true, true)) != CSFFN_OK) return st;
-  if (!aligned16(x) || !aligned16(out)) return CSFFN_ERR_ALIGNMENT;
   const WsLayout L = ws_layout(layer->d, layer->h, B, 0);
-  if ((st = check_ws(ws, ws_bytes, L.ybuf)) != CSFFN_OK) return st;
   FusedArgs a{};
   a.W_gate = layer->w_gate;
   a.W_up = layer->w_up;
@@ -315,6 +330,8 @@ csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x
   cudaStream_t s = as_stream(stream);
   void* xd = at<char>(ws, L.hx);
   void* od = at<char>(ws, L.hout);
+  // the step's own checks, on the staging buffers, before the first copy is issued
+  if ((st = check_cats_step(layer, xd, B, t, idx, a_val, od, ws, ws_bytes)) != CSFFN_OK) return st;
   const size_t xbytes = (size_t)B * layer->d * esize(layer->wdtype);
   const size_t obytes = (size_t)B * layer->d * (out_mode == CSFFN_OUT_BF16 ? 2 : 4);
   if (cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return CSFFN_ERR_CUDA;

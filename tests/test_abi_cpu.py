@@ -146,3 +146,98 @@ def test_kth_rmsnorm_selftest_validation(lib):
     assert s(P(FAKE), BIG, 0, None) == _abi.ERR_INVALID_ARG
     assert s(P(0), BIG, 10, None) == _abi.ERR_WORKSPACE
     assert s(P(FAKE), 16, 10, None) == _abi.ERR_WORKSPACE
+
+
+def test_one_launch_step_validation(lib):
+    """csffn_cats_ffn_forward rejects on the host whatever either of its paths would reject."""
+    def call(L=None, x=FAKE, B=1, t=0.5, cand=None, ccount=None, idx=FAKE, count=FAKE, a_val=FAKE, out=FAKE,
+             mode=_abi.OUT_F32, ws=FAKE, ws_bytes=BIG):
+        L = layer() if L is None else L
+        return lib.csffn_cats_ffn_forward(ctypes.byref(L), P(x), B, t, P(cand), P(ccount), P(idx), P(count),
+                                          P(a_val), P(out), mode, P(ws), ws_bytes, None)
+    assert lib.csffn_cats_ffn_forward(None, P(FAKE), 1, 0.5, None, None, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1,
+                                      P(FAKE), BIG, None) == _abi.ERR_INVALID_ARG
+    assert call(B=17) == _abi.ERR_INVALID_ARG
+    assert call(mode=9) == _abi.ERR_INVALID_ARG
+    assert call(count=0) == _abi.ERR_INVALID_ARG
+    assert call(cand=FAKE) == _abi.ERR_INVALID_ARG  # a list without its count
+    assert call(ccount=FAKE) == _abi.ERR_INVALID_ARG
+    assert call(x=0) == _abi.ERR_INVALID_ARG
+    assert call(idx=0) == _abi.ERR_INVALID_ARG
+    assert call(a_val=0) == _abi.ERR_INVALID_ARG
+    assert call(out=0) == _abi.ERR_INVALID_ARG
+    assert call(t=float("nan")) == _abi.ERR_INVALID_ARG
+    assert call(x=FAKE + 8) == _abi.ERR_ALIGNMENT
+    assert call(out=FAKE + 4) == _abi.ERR_ALIGNMENT
+    no_up = layer()
+    no_up.w_up = None
+    assert call(L=no_up) == _abi.ERR_INVALID_ARG
+    bad_down = layer()
+    bad_down.w_down_t = FAKE + 0x2002
+    assert call(L=bad_down) == _abi.ERR_ALIGNMENT
+    assert call(ws=0) == _abi.ERR_WORKSPACE
+    assert call(ws_bytes=1 << 20) == _abi.ERR_WORKSPACE
+    # shapes the one-launch kernel does not take go to the two-call path, whose own limits hold too
+    assert call(L=layer(d=16384), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
+    assert call(L=layer(d=16384), B=16, idx=0) == _abi.ERR_INVALID_ARG
+    assert call(L=layer(d=4100)) == _abi.ERR_ALIGNMENT
+
+
+def test_host_buffer_step_validation(lib):
+    """csffn_cats_ffn_forward_host validates everything before its first copy (the fake host pointers
+    below are never read)."""
+    def call(L=None, B=1, t=0.5, idx=FAKE, count=FAKE, a_val=FAKE, mode=_abi.OUT_F32, x=FAKE, out=FAKE,
+             ws=FAKE, ws_bytes=BIG):
+        L = layer() if L is None else L
+        return lib.csffn_cats_ffn_forward_host(ctypes.byref(L), P(x), B, t, P(idx), P(count), P(a_val), P(out),
+                                               mode, P(ws), ws_bytes, None)
+    assert call(mode=_abi.OUT_F32_ACCUMULATE) == _abi.ERR_INVALID_ARG  # no accumulation into host memory
+    assert call(B=-1) == _abi.ERR_INVALID_ARG
+    assert call(count=0) == _abi.ERR_INVALID_ARG
+    assert call(x=0) == _abi.ERR_INVALID_ARG
+    assert call(out=0) == _abi.ERR_INVALID_ARG
+    assert call(idx=0) == _abi.ERR_INVALID_ARG
+    assert call(a_val=0) == _abi.ERR_INVALID_ARG
+    assert call(t=float("nan")) == _abi.ERR_INVALID_ARG
+    no_gate = layer()
+    no_gate.w_gate = None
+    assert call(L=no_gate) == _abi.ERR_INVALID_ARG
+    assert call(ws_bytes=1 << 20) == _abi.ERR_WORKSPACE  # the staging buffers are part of the workspace
+    assert call(L=layer(d=16384), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
+
+
+def test_predictor_step_validation(lib):
+    L = layer(act=_abi.ACT_RELU)
+    def call(B=1, rank=256, u=FAKE, v=FAKE, tau=FAKE, t=0.0, idx=FAKE, count=FAKE, a_val=FAKE, out=FAKE,
+             mode=_abi.OUT_F32, ws=FAKE, ws_bytes=BIG, L=L):
+        return lib.csffn_svd_ffn_forward(ctypes.byref(L), P(FAKE), B, rank, P(u), P(v), P(tau), t, P(idx),
+                                         P(count), P(a_val), P(out), mode, P(ws), ws_bytes, None)
+    assert call(B=17) == _abi.ERR_INVALID_ARG
+    assert call(mode=9) == _abi.ERR_INVALID_ARG
+    assert call(count=0) == _abi.ERR_INVALID_ARG
+    assert call(rank=0) == _abi.ERR_INVALID_ARG
+    assert call(rank=5000) == _abi.ERR_INVALID_ARG
+    assert call(rank=100) == _abi.ERR_ALIGNMENT  # rank % 8 (bf16)
+    assert call(u=0) == _abi.ERR_INVALID_ARG
+    assert call(v=0) == _abi.ERR_INVALID_ARG
+    assert call(tau=0) == _abi.ERR_INVALID_ARG
+    assert call(t=float("nan")) == _abi.ERR_INVALID_ARG
+    assert call(v=FAKE + 8) == _abi.ERR_ALIGNMENT
+    assert call(B=8) == _abi.ERR_UNSUPPORTED_SHAPE  # the one-launch kernel takes B <= 4
+    assert call(ws_bytes=1 << 20) == _abi.ERR_WORKSPACE
+
+
+def test_static_entry_validation(lib):
+    def call(L=None, B=1, x=FAKE, idx=FAKE, count=FAKE, a_val=FAKE, out=FAKE, mode=_abi.OUT_F32):
+        L = layer() if L is None else L
+        return lib.csffn_sparse_ffn_forward_static(ctypes.byref(L), P(x), B, P(idx), P(count), P(a_val), P(out),
+                                                   mode, None)
+    assert lib.csffn_sparse_ffn_forward_static(None, P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1,
+                                               None) == _abi.ERR_INVALID_ARG
+    assert call(B=17) == _abi.ERR_INVALID_ARG
+    assert call(mode=9) == _abi.ERR_INVALID_ARG
+    assert call(idx=0) == _abi.ERR_INVALID_ARG
+    assert call(out=FAKE + 4) == _abi.ERR_ALIGNMENT
+    assert call(L=layer(d=4100)) == _abi.ERR_ALIGNMENT
+    assert call(B=8) == _abi.ERR_UNSUPPORTED_SHAPE  # scratch holds B <= 4 at d = 4096
+    assert call(L=layer(d=8192), B=4) == _abi.ERR_UNSUPPORTED_SHAPE
