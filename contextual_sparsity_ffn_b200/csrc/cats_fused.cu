@@ -271,10 +271,15 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   const WT* Wpre = PRED ? reinterpret_cast<const WT*>(p.v_r) : Wg;  // the rows the chunks prefetch
 
   // Rows are positions 0 .. n_rows - 1 of the candidate list (neuron cand_idx[j]) or, without one,
-  // the neurons themselves.  Keep flags and kept activations are stored by position.
+  // the neurons themselves.  Keep flags and kept activations are stored by position.  A candidate
+  // outside 0 .. h - 1 (a malformed list) reads row 0, so every access stays in bounds.
   const int32_t* cand = p.cand_idx;
   const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
-  auto neuron = [&](int j) { return cand ? __ldg(cand + j) : j; };
+  auto neuron = [&](int j) {
+    if (!cand) return j;
+    const int r = __ldg(cand + j);
+    return (unsigned)r < (unsigned)h ? r : 0;
+  };
 
   ChunkMap cm;
   if constexpr (PRED) {
