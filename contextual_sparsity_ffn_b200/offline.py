@@ -6,6 +6,7 @@ SVD "truncation-aware", and Table 3 ablates naive SVD against "+ Data whitening"
 builds both kinds of factors once per layer on the host side (float64 torch linear algebra on
 the weights' device); the decode path then only reads them (csffn_predict_lowrank,
 csffn_svd_ffn_forward, and csffn_calibrate_threshold for the per-neuron thresholds).
+save_artefacts / load_artefacts keep a layer's offline results (thresholds and factors) on disk.
 
 Layout, as the C entry points take it: the gate maps a token row x to x W_gate^T with
 W_gate [h, d] neuron-major, and the predictor computes p = (x U_r) V_r^T + beta with
@@ -23,6 +24,7 @@ from __future__ import annotations
 
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 DEFAULT_RIDGE = 1e-6
@@ -61,3 +63,46 @@ def svd_predictor_factors(w_gate: torch.Tensor, rank: int, x_cal: Optional[torch
     u_rt = u_r.T.to(out_dtype).contiguous()
     v_r = vh[:rank, :].T.to(out_dtype).contiguous()
     return u_rt, v_r
+
+
+# ------------------------------------------------------------------------------ artefacts on disk
+
+def save_artefacts(path: str, **tensors: torch.Tensor) -> None:
+    """Write a layer's offline artefacts (e.g. t, tau, u_rt, v_r) to one .npz file, bit for bit.
+
+    bf16 tensors are stored as their uint16 bit patterns (numpy has no bf16) with the dtype
+    recorded beside them, so load_artefacts gives back identical bits.  Calibration and the SVD
+    run once per model; a decode process reloads their results instead of repeating them.
+    """
+    arrays = {}
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} is not a tensor")
+        c = t.detach().cpu().contiguous()
+        if c.dtype == torch.bfloat16:
+            arrays[name] = c.view(torch.int16).numpy().view(np.uint16)
+            arrays["__dtype__" + name] = np.array("bfloat16")
+        else:
+            arrays[name] = c.numpy()
+            arrays["__dtype__" + name] = np.array(str(c.dtype).replace("torch.", ""))
+    with open(path, "wb") as f:
+        np.savez(f, **arrays)
+
+
+def load_artefacts(path: str, device="cpu") -> dict:
+    """Read a file written by save_artefacts: {name: tensor} with the saved dtypes and bits."""
+    out = {}
+    with np.load(path, allow_pickle=False) as z:
+        for name in z.files:
+            if name.startswith("__dtype__"):
+                continue
+            dt = str(z["__dtype__" + name])
+            a = z[name]
+            if dt == "bfloat16":
+                t = torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16)
+            else:
+                t = torch.from_numpy(a.copy())
+                if str(t.dtype).replace("torch.", "") != dt:
+                    raise ValueError(f"{name}: stored as {a.dtype}, recorded as {dt}")
+            out[name] = t.to(device)
+    return out

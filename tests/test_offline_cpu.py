@@ -131,3 +131,23 @@ def test_whitened_predictor_beats_naive_on_anisotropic_tokens(capsys):
         for r, res in rows:
             print(f"\nr={r}: " + "; ".join(f"{k}: recall {v['recall']:.3f} density {v['density']:.3f} "
                                          f"AUROC {v['auroc']:.3f} rel.err {v['rel_err']:.3f}" for k, v in res.items()))
+
+
+def test_artefacts_round_trip_bit_for_bit(tmp_path):
+    layer = synth.make_layer(35, 0, 32, 48, "bf16", "relu")
+    u_rt, v_r = offline.svd_predictor_factors(_torch_operand(layer.w_gate), 8)
+    tau = torch.linspace(-1.0, 1.0, 48, dtype=torch.float32)
+    t = torch.tensor([0.123456789], dtype=torch.float32)
+    counts = torch.arange(5, dtype=torch.int32)
+    path = str(tmp_path / "layer0.npz")
+    offline.save_artefacts(path, u_rt=u_rt, v_r=v_r, tau=tau, t=t, counts=counts)
+    got = offline.load_artefacts(path)
+    assert set(got) == {"u_rt", "v_r", "tau", "t", "counts"}
+    for name, ref in (("u_rt", u_rt), ("v_r", v_r), ("tau", tau), ("t", t), ("counts", counts)):
+        assert got[name].dtype == ref.dtype and got[name].shape == ref.shape
+        if ref.dtype == torch.bfloat16:
+            assert torch.equal(got[name].view(torch.int16), ref.view(torch.int16))
+        else:
+            assert torch.equal(got[name], ref)
+    with pytest.raises(TypeError):
+        offline.save_artefacts(path, t=0.5)
