@@ -5,7 +5,6 @@ import numpy as np
 import torch
 
 from contextual_sparsity_ffn_b200 import binding as cs
-from contextual_sparsity_ffn_b200 import _abi
 
 DEV = "cuda"
 

@@ -9,7 +9,7 @@ from contextual_sparsity_ffn_b200 import synth
 from contextual_sparsity_ffn_b200 import binding as cs
 from contextual_sparsity_ffn_b200 import _abi
 
-from gpu_helpers import dev, dev_layer, run_dense, run_gate, run_sparse, token_masks
+from gpu_helpers import dev_layer, run_dense, run_gate, run_sparse, token_masks
 
 pytestmark = pytest.mark.gpu
 

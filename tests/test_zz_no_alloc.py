@@ -7,7 +7,6 @@ file checks, through the C ABI, that two calls in a row give the same output as 
 entry point, and that calls too large for the array are refused without a launch.  It is named
 so that pytest collects it last.
 """
-import ctypes
 
 import numpy as np
 import pytest
