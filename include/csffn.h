@@ -208,9 +208,12 @@ csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int 
  *   up and down projections give out.  idx[0 .. *count) = ascending kept neurons, a_val as in
  *   csffn_gate_mask, out as in csffn_sparse_ffn_forward.  The predicted set itself is not written.
  *   u_rt [rank, d], v_r [h, rank] in layer->wdtype, rank % (8 for bf16, 4 for fp32) == 0.
- *   Runs for the shapes csffn_cats_ffn_forward takes in one launch, with the rank's rows beside
- *   them in shared memory; other shapes return CSFFN_ERR_UNSUPPORTED_SHAPE (use the two calls).
- *   ws sized by csffn_workspace_size(layer, B, rank).  B == 0: writes *count = 0. */
+ *   Runs for the shapes csffn_cats_ffn_forward takes in one launch, with a chunk of V_r rows
+ *   (at least 8 rows, at most 64 KB where the rank allows) and y beside them in shared memory;
+ *   other shapes return CSFFN_ERR_UNSUPPORTED_SHAPE (use the two calls).  The mask and a_val are
+ *   bit-for-bit repeatable; out may differ from launch to launch in the last bits, as in
+ *   csffn_cats_ffn_forward.  ws sized by csffn_workspace_size(layer, B, rank).  B == 0: writes
+ *   *count = 0. */
 csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
                                    const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
                                    float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
