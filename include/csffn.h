@@ -64,7 +64,7 @@ extern "C" {
 typedef enum {
   CSFFN_OK = 0,
   CSFFN_ERR_INVALID_ARG = 1,       /* NULL pointer, bad enum, B/n/k/rank out of range */
-  CSFFN_ERR_UNSUPPORTED_SHAPE = 2, /* d/h/B combination this build does not run */
+  CSFFN_ERR_UNSUPPORTED_SHAPE = 2, /* d/h/B combination the library does not run */
   CSFFN_ERR_ALIGNMENT = 3,         /* d not a multiple of the vector width, or pointer not 16-B aligned */
   CSFFN_ERR_WORKSPACE = 4,         /* ws NULL or ws_bytes below the queried size */
   CSFFN_ERR_CUDA = 5,              /* a CUDA runtime call or kernel launch failed */
