@@ -48,7 +48,8 @@ RMS_EPS = 1e-6
 
 
 def decode(a) -> np.ndarray:
-    """Exact float64 value of a stored operand: bf16 bit patterns (uint16) or float32."""
+    """Exact float64 value of a stored operand: bf16 bit patterns (uint16) or float32 (operand
+    decoding, no passage of the method)."""
     a = np.asarray(a)
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
@@ -56,7 +57,8 @@ def decode(a) -> np.ndarray:
 
 
 def silu(z: np.ndarray) -> np.ndarray:
-    """SiLU(z) = z * sigmoid(z) = z / (1 + e^{-z}) (the SwiGLU gate activation)."""
+    """SiLU(z) = z * sigmoid(z) = z / (1 + e^{-z}): the SwiGLU gate activation whose output
+    [CATS] (abstract) thresholds."""
     with np.errstate(over="ignore"):
         return z / (1.0 + np.exp(-z))
 
@@ -67,6 +69,7 @@ def relu(z: np.ndarray) -> np.ndarray:
 
 
 def activation(z: np.ndarray, act: str) -> np.ndarray:
+    """The layer's gate activation: SiLU ([CATS] abstract, SwiGLU) or ReLU ([SVDP] abstract, ReGLU)."""
     if act == "silu":
         return silu(z)
     if act == "relu":
@@ -80,7 +83,9 @@ def _tokens(x) -> np.ndarray:
 
 
 def gate_preactivation(x, layer) -> np.ndarray:
-    """z[b, i] = x_b . W_gate[i, :] + beta_i  ->  [B, h]."""
+    """The gate projection ([CATS] abstract: the gate GEMV; [SVDP] Fig. 3: the gate of the
+    predicted neurons): z[b, i] = x_b . W_gate[i, :] + beta_i  ->  [B, h].  beta is the explicit
+    per-neuron gate bias of the ReGLU workload (a reading; absent elsewhere)."""
     z = _tokens(x) @ decode(layer.w_gate).T
     if layer.bias is not None:
         z = z + decode(layer.bias)[None, :]
@@ -88,17 +93,20 @@ def gate_preactivation(x, layer) -> np.ndarray:
 
 
 def gate_activation(x, layer) -> np.ndarray:
-    """a = act(z): SiLU for SwiGLU, ReLU for ReGLU  ->  [B, h]."""
+    """a = act(z) ([CATS] abstract: the activation that is thresholded): SiLU for SwiGLU, ReLU
+    for ReGLU  ->  [B, h]."""
     return activation(gate_preactivation(x, layer), layer.act)
 
 
 def up_projection(x, layer) -> np.ndarray:
-    """u[b, i] = x_b . W_up[i, :]  ->  [B, h]."""
+    """The up projection ([CATS] abstract: the flag-gated GEMV reads only the kept rows;
+    [SVDP] Fig. 3: up runs after the gate): u[b, i] = x_b . W_up[i, :]  ->  [B, h]."""
     return _tokens(x) @ decode(layer.w_up).T
 
 
 def down_projection(g: np.ndarray, layer) -> np.ndarray:
-    """out[b, :] = sum_i g[b, i] * W_down^T[i, :]  ->  [B, d]."""
+    """The down projection over the gated activations ([CATS] abstract; [SVDP] Fig. 3):
+    out[b, :] = sum_i g[b, i] * W_down^T[i, :]  ->  [B, d]."""
     return g @ decode(layer.w_down_t)
 
 
@@ -117,7 +125,8 @@ def cats_mask(a: np.ndarray, t: float) -> np.ndarray:
 
 
 def sparse_ffn(x, layer, mask: np.ndarray) -> np.ndarray:
-    """The dense FFN evaluated with the activations outside ``mask`` set to zero.
+    """The dense FFN evaluated with the activations outside ``mask`` set to zero ([CATS]
+    abstract: sub-threshold activations are zeroed, so their rows contribute nothing).
 
     ``mask`` is [B, h] (or [h], broadcast over tokens).  This is the result the
     sparse executor must reach by reading only the active rows.
@@ -136,17 +145,22 @@ def cats_ffn(x, layer, t: float) -> tuple:
 
 
 def union_mask(mask: np.ndarray) -> np.ndarray:
-    """Rows a small batch must read: the union over tokens of the per-token masks -> [h]."""
+    """Rows a small batch must read: the union over tokens of the per-token masks -> [h].
+
+    The pages treat one token at a time; the reading for a batch is that the union selects the
+    rows that are read while every token keeps its own values."""
     return np.asarray(mask, dtype=bool).reshape(-1, np.shape(mask)[-1]).any(axis=0)
 
 
 def active_indices(row_mask: np.ndarray) -> np.ndarray:
-    """Ascending int32 indices of the set entries of a [h] mask."""
+    """Ascending int32 indices of the set entries of a [h] mask (the index-order reading: the
+    pages fix no order)."""
     return np.flatnonzero(np.asarray(row_mask, dtype=bool)).astype(np.int32)
 
 
 def order_statistic_rank(s: float, m: int) -> int:
-    """k = ceil(s * m), clamped to [0, m].
+    """k = ceil(s * m), clamped to [0, m]: the rank of the lower order statistic that the
+    quantile reading of the calibrated threshold ([CATS] abstract; [SVDP] Fig. 1) selects.
 
     s is first taken at float32 precision (the type the library interface
     carries), then the product is evaluated exactly; 0.9 of 50 values is 45.
@@ -156,7 +170,8 @@ def order_statistic_rank(s: float, m: int) -> int:
 
 
 def calibrate_global(x_cal, layer, s: float) -> float:
-    """One CATS threshold per layer: the s-quantile of |a| pooled over calibration set x neurons.
+    """One CATS threshold per layer ([CATS] abstract: a threshold set for a target sparsity):
+    the s-quantile of |a| pooled over calibration set x neurons.
 
     M = N*h values |a|, sorted ascending; k = ceil(s*M); t = v_(k) (1-indexed),
     t = 0 when k = 0.  On the calibration set #{|a| <= t} >= k, with equality
@@ -168,7 +183,8 @@ def calibrate_global(x_cal, layer, s: float) -> float:
 
 
 def kth_smallest(values: np.ndarray, k: int) -> float:
-    """v_(k) of a flat array (1-indexed); used for checking order-statistic selection."""
+    """v_(k) of a flat array (1-indexed); used for checking order-statistic selection (no
+    passage of the method: the check of the selection behind the quantile reading)."""
     v = np.sort(np.asarray(values, dtype=np.float64).ravel())
     return float(v[k - 1])
 
@@ -232,7 +248,8 @@ def calibrate_per_neuron(x_cal, u_rt, v_r, bias, q: float) -> np.ndarray:
 
 
 def predicted_mask(p: np.ndarray, tau: np.ndarray) -> np.ndarray:
-    """P = {i : p_i > tau_i} per token -> [B, h]."""
+    """[SVDP] Fig. 1 and Fig. 2: a neuron is predicted active when its predictor output exceeds
+    its calibrated threshold, P = {i : p_i > tau_i} per token -> [B, h]."""
     return p > np.asarray(tau, dtype=np.float64)[None, :]
 
 
@@ -251,7 +268,9 @@ def reglu_sequential(x, layer, pred_mask: np.ndarray) -> tuple:
 
 
 def rmsnorm(v: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
-    """RMSNorm with unit gain: v / sqrt(mean(v^2) + eps), per row."""
+    """RMSNorm with unit gain: v / sqrt(mean(v^2) + eps), per row.  The input step of the
+    decoder blocks whose FFN shapes [SVDP] Table 12 lists; the pages do not print it (reading:
+    unit gain, eps = 1e-6)."""
     v = np.asarray(v, dtype=np.float64)
     return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
 
@@ -259,7 +278,8 @@ def rmsnorm(v: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
 def round_to_bf16(v: np.ndarray) -> np.ndarray:
     """Value of v after rounding to bfloat16 (nearest, ties to even), as float64.
 
-    Done through PyTorch's CPU cast, independently of the input encoder.
+    Done through PyTorch's CPU cast, independently of the input encoder.  The bf16 rounding of the
+    FFN input is a reading (the pages run bf16 models but print no rounding step).
     """
     import torch
 
@@ -268,7 +288,8 @@ def round_to_bf16(v: np.ndarray) -> np.ndarray:
 
 
 def stack_layer(h: np.ndarray, layer, t=None, mask=None) -> tuple:
-    """One residual block of the FFN stack: h + FFN(bf16(RMSNorm(h))).
+    """One residual block of the FFN stack: h + FFN(bf16(RMSNorm(h))) (the decoder block around
+    the FFN of the models the pages evaluate; the stack itself is a harness, not a page's method).
 
     With ``mask`` the FFN is the sparse one on that mask; with ``t`` the CATS
     mask at t; with neither, the dense FFN.  Returns (h_next, xn, mask_used).
@@ -296,7 +317,8 @@ def sirius_round(x_steps, layer, t: float) -> tuple:
 
 
 def rel_l2(y, y_ref) -> float:
-    """max over vectors of ||y - y_ref||_2 / ||y_ref||_2 (0/0 counts as 0)."""
+    """max over vectors of ||y - y_ref||_2 / ||y_ref||_2 (0/0 counts as 0): the parity measure,
+    no passage of the method."""
     y = np.atleast_2d(np.asarray(y, dtype=np.float64))
     r = np.atleast_2d(np.asarray(y_ref, dtype=np.float64))
     num = np.linalg.norm(y - r, axis=-1)
