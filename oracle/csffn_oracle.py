@@ -182,13 +182,6 @@ def calibrate_global(x_cal, layer, s: float) -> float:
     return 0.0 if k == 0 else float(v[k - 1])
 
 
-def kth_smallest(values: np.ndarray, k: int) -> float:
-    """v_(k) of a flat array (1-indexed); used for checking order-statistic selection (no
-    passage of the method: the check of the selection behind the quantile reading)."""
-    v = np.sort(np.asarray(values, dtype=np.float64).ravel())
-    return float(v[k - 1])
-
-
 def svd_factors(w_gate, r: int) -> tuple:
     """[SVDP] abstract / Fig. 1: rank-r truncated SVD of the gate projection.
 

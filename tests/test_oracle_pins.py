@@ -241,9 +241,29 @@ def test_per_neuron_calibration_matches_numpy():
     for q in [0.5, 0.9]:
         tau = oracle.calibrate_per_neuron(xc, urt, vr, beta, q)
         np.testing.assert_array_equal(tau, np.quantile(p, q, axis=0, method="inverted_cdf"))
-        frac = (p > tau[None, :]).mean(axis=0)
+        frac = oracle.predicted_mask(p, tau).mean(axis=0)
         assert np.all(frac <= 1 - q + 1e-12)
     assert np.all(np.isneginf(oracle.calibrate_per_neuron(xc, urt, vr, beta, 0.0)))
+
+
+def test_predicted_mask_brute_force():
+    """[SVDP] Fig. 1 and Fig. 2: token b predicts neuron i iff p[b, i] > tau_i (strict), with tau
+    per neuron (broadcast over tokens).  A non-square case (B = 3 tokens, h = 5 neurons) with a tie
+    p == tau (inactive), a negative tau (a negative p above it is active) and tau = -inf (always
+    active, the k = 0 calibration), against a Python loop and a table written out by hand."""
+    p = np.array([[0.5, -1.0, 2.0, 0.0, 3.0],
+                  [1.0, -2.0, -0.5, -1e300, -9.0],
+                  [0.2, 0.2, 0.2, 0.2, 0.2]])
+    tau = np.array([0.5, -1.5, 1.0, -np.inf, 0.2])
+    loop = [[p[b][i] > tau[i] for i in range(5)] for b in range(3)]
+    by_hand = [[False, True, True, True, True],
+               [True, False, False, True, False],
+               [False, True, False, True, False]]
+    got = oracle.predicted_mask(p, tau)
+    assert got.shape == (3, 5) and got.dtype == bool
+    assert got.tolist() == loop == by_hand
+    # one token: the [1, h] row of the same rule
+    assert oracle.predicted_mask(p[1:2], tau).tolist() == [by_hand[1]]
 
 
 # ----------------------------------------------------------------------------- SVD
@@ -392,6 +412,7 @@ PIN_TESTS = [
     lambda: test_whitened_svd_is_the_best_rank_r_fit_on_calibration(),
     lambda: test_whitened_svd_full_rank_and_isotropic_data(),
     lambda: test_silu_matches_scipy_expit(),
+    lambda: test_predicted_mask_brute_force(),
 ]
 
 
@@ -440,6 +461,18 @@ def _mut_whiten_not_mapped_back(w_gate, r, x_cal, ridge=oracle.WHITEN_RIDGE):
     return (u[:, :r] * s[None, :r]).T.copy(), vt[:r, :].T.copy()
 
 
+def _mut_pred_ge(p, tau):
+    return p >= np.asarray(tau, dtype=np.float64)[None, :]
+
+
+def _mut_pred_tau_negated(p, tau):
+    return p > -np.asarray(tau, dtype=np.float64)[None, :]
+
+
+def _mut_pred_tau_token_axis(p, tau):
+    return p > np.asarray(tau, dtype=np.float64)[:, None]
+
+
 def _mut_up_uses_gate(x, layer):
     return oracle.csffn_oracle._tokens(x) @ oracle.decode(layer.w_gate).T
 
@@ -462,6 +495,9 @@ MUTANTS = {
     "whiten_not_mapped_back": ("svd_factors_whitened", _mut_whiten_not_mapped_back),
     "up_uses_gate": ("up_projection", _mut_up_uses_gate),
     "reglu_ignores_pred": ("reglu_sequential", _mut_reglu_ignores_pred),
+    "pred_ge": ("predicted_mask", _mut_pred_ge),
+    "pred_tau_negated": ("predicted_mask", _mut_pred_tau_negated),
+    "pred_tau_token_axis": ("predicted_mask", _mut_pred_tau_token_axis),
 }
 
 
