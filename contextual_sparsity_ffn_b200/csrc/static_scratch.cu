@@ -14,9 +14,14 @@
 // the only part that must start at zero, are cleared on the caller's stream before each launch.
 //
 // Host code cannot use the array's name as a device address (in host code it names a host-side
-// stand-in), so the device address is looked up once per device with cudaGetSymbolAddress, with
-// that device current, on the first call made on it.  Because that first call does this set-up,
-// it should come before any stream capture that includes the entry point.
+// stand-in), so the device address is looked up with cudaGetSymbolAddress, with the device
+// current, on the first call made on it.  Because that first call does this set-up, it should
+// come before any stream capture that includes the entry point.  The address is remembered per
+// device together with the CUDA context it belongs to: after a device reset (a new context, where
+// the array may sit at another address) the next call looks it up again instead of using the old
+// one.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -30,22 +35,50 @@ static __device__ __align__(256) unsigned char g_static_scratch[CSFFN_STATIC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchAddress {
+  CUcontext ctx;  // the context the address was looked up in
+  void* ptr;
+};
+ScratchAddress g_scratch[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device (looked up once per device).
+// cuCtxGetCurrent from the driver, through the runtime (no link against libcuda).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_getter() {
+  static CtxGetCurrentFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }();
+  return fn;
+}
+
+CUcontext current_context() {
+  CUcontext c = nullptr;
+  CtxGetCurrentFn get = ctx_getter();
+  if (!get || get(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_static_scratch on the current device: looked up once per device and
+// context, with the device current.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  CUcontext ctx = current_context();
+  if (g_scratch[dev].ptr == nullptr || ctx == nullptr || g_scratch[dev].ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // makes the device's context current if none was
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    g_scratch[dev].ptr = p;
+    g_scratch[dev].ctx = current_context();
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return cudaSuccess;
 }
 

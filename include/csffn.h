@@ -270,7 +270,9 @@ csffn_status csffn_selftest_timeout(void* ws, size_t ws_bytes, int spin_limit, v
  *   threads) race, so order them on one stream.  The reduction counters are cleared on `stream`
  *   before each launch; the rest of the array is fully rewritten before it is read.
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress with
- *   that device current); make that first call before any stream capture that includes it.
+ *   that device current); make that first call before any stream capture that includes it.  The
+ *   address is kept per device and CUDA context, so after a device reset the next call (again
+ *   outside a capture) looks it up anew.
  *   Other arguments, layouts and errors as csffn_sparse_ffn_forward. */
 #define CSFFN_STATIC_SCRATCH_BYTES (8u << 20)
 csffn_status csffn_sparse_ffn_forward_static(const csffn_layer* layer, const void* x, int B,

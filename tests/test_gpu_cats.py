@@ -240,6 +240,15 @@ def test_dense_token_block_tensor_cores(d, h, B, act):
 
 # ------------------------------------------------------------------------------ one-launch decode step
 
+def check_values(a_val, idx, a_ref, m, t):
+    """a_val against the oracle's activations, element by element: a where the token keeps the row,
+    0 where it rejects it; the per-token masks agree with the oracle's outside the band."""
+    tb = np.abs(np.abs(a_ref) - t) < 1e-3 * abs(t)
+    assert np.array_equal(m[~tb], oracle.cats_mask(a_ref, t)[~tb])
+    np.testing.assert_allclose(a_val, np.where(m, a_ref, 0.0)[:, idx], rtol=1e-4,
+                               atol=1e-6 * np.abs(a_ref).max())
+
+
 def run_fused(layer, x_np, t, out_dtype=torch.float32, ws=None):
     x = dev(x_np if x_np.ndim == 2 else x_np[None, :])
     B = x.shape[0]
@@ -273,6 +282,7 @@ def test_fused_decode_matches_oracle_and_two_call_path(d, h, B, dtype, s):
     got[idx] = True
     assert np.array_equal(got[~band], oracle.union_mask(oracle.cats_mask(a_ref, t))[~band])
     m = token_masks(idx, a_val, h)
+    check_values(a_val, idx, a_ref, m, t)
     tol = TOL_F32 if dtype == "f32" else TOL_BF16_F32OUT
     assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= tol
     # the two-call path (other kernels, other summation order) gives the same set outside the band,
@@ -339,6 +349,8 @@ def test_fused_decode_reglu_with_gate_bias():
         got[idx] = True
         assert np.array_equal(got[~band], oracle.union_mask(oracle.cats_mask(a_ref, t))[~band])
         m = token_masks(idx, a_val, spec.h)
+        if t > 0:
+            check_values(a_val, idx, a_ref, m, t)
         assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= TOL_BF16_F32OUT
 
 
@@ -362,12 +374,14 @@ def test_fused_decode_7b_low_threshold_keeps_negative_activations():
         got[idx] = True
         assert np.array_equal(got[~band], keep_ref[~band])
         m = token_masks(idx, a_val, spec.h)
+        check_values(a_val, idx, a_ref, m, t)
         assert oracle.rel_l2(out, oracle.sparse_ffn(x, spec, m)) <= TOL_BF16_F32OUT
 
 
 def test_fused_decode_host_buffers():
-    """csffn_cats_ffn_forward_host: tokens in and output out through pinned host memory give the
-    device entry point's result (bf16 and fp32 outputs)."""
+    """csffn_cats_ffn_forward_host: tokens in and output out through pinned host memory, checked
+    against the oracle on the call's own mask, and against the device entry point's result (bf16
+    and fp32 outputs)."""
     spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=64)
     t = oracle.calibrate_global(xc, spec, 0.5)
     layer = dev_layer(spec)
@@ -383,5 +397,14 @@ def test_fused_decode_host_buffers():
         torch.cuda.synchronize()
         assert cs.check_status(ws) == 0
         n = int(cnt.item())
-        assert np.array_equal(idx[:n].cpu().numpy(), idx_d)
-        assert oracle.rel_l2(oh.float().numpy().astype(np.float64), out_d) <= tol
+        got_idx = idx[:n].cpu().numpy()
+        got_av = av[:, :n].cpu().numpy().astype(np.float64)
+        assert_index_list(got_idx, spec.h)
+        m = token_masks(got_idx, got_av, spec.h)
+        a_ref = oracle.gate_activation(x, spec)
+        check_values(got_av, got_idx, a_ref, m, t)
+        got = oh.float().numpy().astype(np.float64)
+        ref = oracle.sparse_ffn(x, spec, m)
+        assert oracle.rel_l2(got, ref) <= (TOL_BF16_F32OUT if dtype == torch.float32 else TOL_BF16)
+        assert np.array_equal(got_idx, idx_d)
+        assert oracle.rel_l2(got, out_d) <= tol
