@@ -260,6 +260,23 @@ def reglu_sequential(x, layer, pred_mask: np.ndarray) -> tuple:
     return out, a_mask
 
 
+def reglu_parallel(x, layer, pred_mask: np.ndarray) -> tuple:
+    """[SVDP] Table 2 caption ("r=1024 parallel") and Table 3 ("Parallel pipeline"): the gate and
+    the up projection both run on the predicted set P (neither waits for the other); the down
+    projection takes their gated product ReLU(z_i) * u_i, which is zero outside
+    A = {i in P : z_i > 0}.  The pages name the pipeline without a formula; this is the reading.
+
+    Returns (out [B, d], A [B, h]).  ``pred_mask`` is per token [B, h] or [h].  The output is the
+    sequential pipeline's (the pipelines differ in which rows they read, not in what they compute).
+    """
+    z = gate_preactivation(x, layer)
+    p = np.asarray(pred_mask, dtype=bool)
+    if p.ndim == 1:
+        p = np.broadcast_to(p[None, :], z.shape)
+    g = np.where(p, relu(z) * up_projection(x, layer), 0.0)
+    return down_projection(g, layer), p & (z > 0.0)
+
+
 def rmsnorm(v: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
     """RMSNorm with unit gain: v / sqrt(mean(v^2) + eps), per row.  The input step of the
     decoder blocks whose FFN shapes [SVDP] Table 12 lists; the pages do not print it (reading:
@@ -298,15 +315,46 @@ def sirius_round(x_steps, layer, t: float) -> tuple:
     """[SIRIUS] "Approach", FFN part only: the sparse FFN drafts each of the chunk's
     tokens one at a time, then the dense FFN verifies the whole chunk in one batch.
 
+    Each draft uses only its own token's mask, so the T drafts are evaluated together as T
+    independent rows (the batched CATS FFN keeps per-token masks and values).
     Returns (sparse outputs [T, d], dense outputs [T, d], masks [T, h]).
     """
     x = _tokens(x_steps)
-    sparse, masks = [], []
-    for b in range(x.shape[0]):
-        o, m = cats_ffn(x[b], layer, t)
-        sparse.append(o[0])
-        masks.append(m[0])
-    return np.stack(sparse), dense_ffn(x, layer), np.stack(masks)
+    sparse, masks = cats_ffn(x, layer, t)
+    return sparse, dense_ffn(x, layer), masks
+
+
+def round_effective_density(masks: np.ndarray) -> dict:
+    """[SIRIUS] "Key results" (effective density) and "Approach" (the full model verifies the
+    chunk in parallel), FFN weights only.  The pages give the figure but not its formula; reading:
+    weight rows a round reads over the rows T dense decode steps read.
+
+    A draft of token t reads all h rows of W_gate and the W_up and W_down^T rows of its kept set
+    (n_t rows each); the verify reads all 3h rows once for the whole chunk; T dense decode steps
+    read 3h rows each.  Every draft is counted as accepted (no model, so no rejection: the average
+    advance length is T).  ``masks``: the drafts' keep masks [T, h].
+    Returns {"neuron_density": mean_t n_t / h, "effective_density": (sum_t (h + 2 n_t) + 3h) / (3 h T)}.
+    """
+    m = np.asarray(masks, dtype=bool)
+    T, h = m.shape
+    n = m.sum(axis=1).astype(np.float64)
+    return {"neuron_density": float(n.mean() / h),
+            "effective_density": float((np.sum(h + 2.0 * n) + 3.0 * h) / (3.0 * h * T))}
+
+
+def draft_agreement(sparse_out: np.ndarray, dense_out: np.ndarray, proj: np.ndarray) -> dict:
+    """Agreement of the sparse drafts with the dense verify over a round ([SIRIUS] "Approach": the
+    full model verifies the sparse model's tokens).  Without a language-model head, a fixed matrix
+    ``proj`` [d, V] stands in for it (a reading): token t agrees when the arg max over V of
+    sparse_t . proj equals that of dense_t . proj (first index on ties).
+    Returns {"rel_l2": [T] per-token ||s_t - d_t|| / ||d_t||, "top1": [T] bool}.
+    """
+    s = np.atleast_2d(np.asarray(sparse_out, dtype=np.float64))
+    dn = np.atleast_2d(np.asarray(dense_out, dtype=np.float64))
+    r = np.asarray(proj, dtype=np.float64)
+    rel = np.linalg.norm(s - dn, axis=1) / np.linalg.norm(dn, axis=1)
+    top1 = np.argmax(s @ r, axis=1) == np.argmax(dn @ r, axis=1)
+    return {"rel_l2": rel, "top1": top1}
 
 
 def rel_l2(y, y_ref) -> float:

@@ -193,6 +193,43 @@ def test_reglu_sequential_brute_force():
     np.testing.assert_allclose(out, bf_dense_ffn(x, layer, pred=pred), rtol=1e-12, atol=1e-15)
 
 
+def test_reglu_parallel_brute_force():
+    """[SVDP] Table 2 caption / Table 3 "Parallel pipeline": gate and up on P, the product ReLU(z) u
+    on P into the down projection: per-element loops, and the active set A = P & (z > 0)."""
+    d, h = 24, 30
+    s = synth.reglu_bias_sigma(d)
+    layer = _tiny_layer(d, h, act="relu", bias=(-1.5 * s, 0.5 * s))
+    x = _tiny_tokens(3, d)
+    pred = np.random.default_rng(4).random((3, h)) < 0.5
+    out, amask = oracle.reglu_parallel(x, layer, pred)
+    np.testing.assert_array_equal(amask, pred & (bf_activations(x, layer) > 0))
+    np.testing.assert_allclose(out, bf_dense_ffn(x, layer, pred=pred), rtol=1e-12, atol=1e-15)
+    # one shared predicted set ([h]) is every token's
+    out1, _ = oracle.reglu_parallel(x, layer, pred[0])
+    np.testing.assert_allclose(out1, bf_dense_ffn(x, layer, pred=np.broadcast_to(pred[0], (3, h))),
+                               rtol=1e-12, atol=1e-15)
+
+
+def test_round_effective_density_by_hand():
+    """[SIRIUS] "Key results" / "Approach", FFN weights: (sum_t (h + 2 n_t) + 3 h) / (3 h T)."""
+    m = np.array([[1, 0, 0, 0], [1, 1, 1, 0]], bool)  # T = 2, h = 4, n = (1, 3)
+    r = oracle.round_effective_density(m)
+    assert r["neuron_density"] == 0.5
+    assert r["effective_density"] == pytest.approx(28.0 / 24.0, rel=1e-15)  # (6 + 10 + 12) / 24
+    T, h = 16, 10
+    assert oracle.round_effective_density(np.ones((T, h), bool))["effective_density"] == pytest.approx(1 + 1 / T)
+    assert oracle.round_effective_density(np.zeros((T, h), bool))["effective_density"] == pytest.approx(1 / 3 + 1 / T)
+
+
+def test_draft_agreement_by_hand():
+    proj = np.array([[1.0, 0.0, 0.0], [0.0, 1.0, 0.0]])  # d = 2, V = 3
+    sp = np.array([[2.0, 1.0], [0.0, 3.0]])
+    de = np.array([[2.0, 0.0], [1.0, 0.0]])
+    r = oracle.draft_agreement(sp, de, proj)
+    assert r["top1"].tolist() == [True, False]  # arg max 0 vs 0; 1 vs 0
+    np.testing.assert_allclose(r["rel_l2"], [0.5, math.sqrt(10.0)], rtol=1e-15)
+
+
 def test_calibration_exhaustive_count():
     d, h, n = 16, 24, 10
     layer = _tiny_layer(d, h)
@@ -413,6 +450,9 @@ PIN_TESTS = [
     lambda: test_whitened_svd_full_rank_and_isotropic_data(),
     lambda: test_silu_matches_scipy_expit(),
     lambda: test_predicted_mask_brute_force(),
+    lambda: test_reglu_parallel_brute_force(),
+    lambda: test_round_effective_density_by_hand(),
+    lambda: test_draft_agreement_by_hand(),
 ]
 
 
@@ -484,6 +524,31 @@ def _mut_reglu_ignores_pred(x, layer, pred_mask):
     return out, a_mask
 
 
+def _mut_parallel_ignores_pred(x, layer, pred_mask):
+    z = oracle.gate_preactivation(x, layer)
+    g = oracle.relu(z) * oracle.up_projection(x, layer)
+    return oracle.down_projection(g, layer), z > 0.0
+
+
+def _mut_parallel_no_relu(x, layer, pred_mask):
+    z = oracle.gate_preactivation(x, layer)
+    p = np.broadcast_to(np.asarray(pred_mask, bool), z.shape)
+    return oracle.down_projection(np.where(p, z * oracle.up_projection(x, layer), 0.0), layer), p & (z > 0)
+
+
+def _mut_density_no_verify(masks):
+    m = np.asarray(masks, dtype=bool)
+    T, h = m.shape
+    n = m.sum(axis=1).astype(np.float64)
+    return {"neuron_density": float(n.mean() / h), "effective_density": float(np.sum(h + 2.0 * n) / (3.0 * h * T))}
+
+
+def _mut_agreement_argmin(sparse_out, dense_out, proj):
+    s, dn, r = (np.atleast_2d(np.asarray(v, dtype=np.float64)) for v in (sparse_out, dense_out, proj))
+    return {"rel_l2": np.linalg.norm(s - dn, axis=1) / np.linalg.norm(dn, axis=1),
+            "top1": np.argmin(s @ r, axis=1) == np.argmin(dn @ r, axis=1)}
+
+
 MUTANTS = {
     "silu_sign": ("silu", _mut_silu_sign),
     "dropped_bias": ("gate_preactivation", _mut_no_bias),
@@ -498,6 +563,10 @@ MUTANTS = {
     "pred_ge": ("predicted_mask", _mut_pred_ge),
     "pred_tau_negated": ("predicted_mask", _mut_pred_tau_negated),
     "pred_tau_token_axis": ("predicted_mask", _mut_pred_tau_token_axis),
+    "parallel_ignores_pred": ("reglu_parallel", _mut_parallel_ignores_pred),
+    "parallel_no_relu": ("reglu_parallel", _mut_parallel_no_relu),
+    "density_no_verify": ("round_effective_density", _mut_density_no_verify),
+    "agreement_argmin": ("draft_agreement", _mut_agreement_argmin),
 }
 
 
