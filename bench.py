@@ -27,7 +27,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -47,7 +46,9 @@ N_TOKENS = 64
 # Headline path: the one-launch csffn_cats_ffn_forward; the two-call path (csffn_gate_mask +
 # csffn_sparse_ffn_forward, same outputs) is reported beside it.
 HEADLINE_TWO_CALL = False
-PROFILE_SUMMARY = os.path.join(HERE, "profiles", "cats_fused_llama2_7b_b1.md")
+# The machine-read figures of the headline kernel's ncu capture (the summary beside it is for people).
+PROFILE_JSON = os.path.join(HERE, "profiles", "cats_ring_llama2_7b_b1.json")
+TIMED_REPLAYS = 9  # replays of the K-step graph; the headline is their median
 
 
 def parse_args(argv=None):
@@ -171,7 +172,7 @@ def measured_hbm_gbs():
 
 
 # Sources of the headline kernel: the profiled traffic is reported only while these are unchanged.
-PROFILED_SOURCES = ("cats_fused.cu", "common.cuh", "gemv.cuh", "tma.cuh", "kernels.h")
+PROFILED_SOURCES = ("ring.cu", "fused_end.cuh", "common.cuh", "tma.cuh", "kernels.h")
 
 
 def csrc_hash() -> str:
@@ -184,17 +185,16 @@ def csrc_hash() -> str:
 
 
 def profiled_traffic():
-    """dram bytes per headline-kernel launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes (read + write) per headline-kernel launch from the committed ncu figures, if they
+    were taken on this source."""
     try:
-        with open(PROFILE_SUMMARY) as f:
-            text = f.read()
-    except OSError:
+        with open(PROFILE_JSON) as f:
+            rec = json.load(f)
+        traffic = float(rec["traffic_bytes_per_launch"])
+        captured = str(rec["csrc_sha256_16"])
+    except (OSError, ValueError, KeyError, TypeError):
         return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    hsh = re.search(r"csrc_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not hsh or hsh.group(1) != csrc_hash():
-        return None
-    return float(m.group(1))
+    return traffic if captured == csrc_hash() else None
 
 
 # ---------------------------------------------------------------------------------- csffn arm
@@ -379,22 +379,32 @@ def csffn_arm(args, world, rank, local):
         li = k % N_ROT
         cs.dense_ffn_forward(layers[li], xs[k % N_TOKENS: k % N_TOKENS + 1], out, buf.ws)
 
-    def time_graph(g, replays_warm):
+    spread = {}
+
+    def time_graph(g, replays_warm, key=None):
+        """Median over TIMED_REPLAYS replays of the K-step graph (ms per replay); each replay is
+        bracketed by a barrier and a device synchronise, and timed by events on the capture stream."""
         for _ in range(replays_warm):
             g.replay()
         torch.cuda.synchronize()
+        times = []
+        for _ in range(TIMED_REPLAYS):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record()
+                g.replay()
+                e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
         if world > 1:
             dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record()
-            g.replay()
-            e1.record()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return e0.elapsed_time(e1)
+        if key is not None:
+            spread[key] = {"replays": len(times), "min_ms": round(min(times), 5),
+                           "median_ms": round(statistics.median(times), 5), "max_ms": round(max(times), 5)}
+        return statistics.median(times)
 
     # ---- main measurement: K steps at the headline sparsity in one graph, events around the replay.
     # No event nodes inside this graph: they add a gap before every launch.  With the one-launch path
@@ -408,7 +418,7 @@ def csffn_arm(args, world, rank, local):
     while time.time() < t_end:
         g_main.replay()
         torch.cuda.synchronize()
-    ms = time_graph(g_main, warm_replays)
+    ms = time_graph(g_main, warm_replays, key="headline")
     clocks = sampler.stop()
     ms_max = max_over_ranks(ms, world, dev)
     if HEADLINE_TWO_CALL:
@@ -449,7 +459,7 @@ def csffn_arm(args, world, rank, local):
         kern_name = "gate_stream_kernel (csffn_gate_mask)"
         kern_bytes = 2.0 * H * D + 2 * D + 8.0 * n_act
     else:
-        kern_name = "cats_fused_kernel (csffn_cats_ffn_forward)"
+        kern_name = "cats_ring_kernel (csffn_cats_ffn_forward)"
         kern_bytes = step_bytes(n_act)  # the whole step is one kernel launch
     kern_gbs = kern_bytes / (kern_avg_us * 1e-6) / 1e9
 
@@ -510,7 +520,8 @@ def csffn_arm(args, world, rank, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"inputs larger than L2: steps rotate over {N_ROT} layer weight sets "
                          f"({N_ROT * 3 * 2 * H * D / 1e9:.2f} GB)",
-                   "timing": "K steps in one CUDA graph, CUDA events on the capture stream, max over ranks"},
+                   "timing": f"K steps in one CUDA graph, CUDA events on the capture stream, median of "
+                             f"{TIMED_REPLAYS} replays, max over ranks"},
         "tokens_per_s": round(world * K / (ms_max * 1e-3), 1),
         "active_rows": round(n_act, 1),
         "bytes_needed_mb": round(step_bytes(n_act) / 1e6, 2),
@@ -524,7 +535,8 @@ def csffn_arm(args, world, rank, local):
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": round(kern_bytes),
                      "avg_launch_us": round(kern_avg_us, 3),
                      "timing": ("events around each csffn_gate_mask launch inside a graph" if HEADLINE_TWO_CALL else
-                                "events around the timed K-launch graph replay; per launch = total / K")},
+                                "events around each replay of the K-launch graph; per launch = median replay / K"),
+                     "replays": spread.get("headline")},
         "e2e": e2e,
         "gpu_launches": (3 if HEADLINE_TWO_CALL else 1) * K,
         "clocks": clocks,

@@ -213,7 +213,7 @@ csffn_status check_cats_step(const csffn_layer* layer, const void* x, int B, flo
   csffn_status st = check_weights(layer, true, true, true);
   if (st != CSFFN_OK) return st;
   if (!aligned16(x) || !aligned16(out)) return CSFFN_ERR_ALIGNMENT;
-  if (!cats_fused_supported(layer->d, B, layer->wdtype) &&
+  if (!cats_ring_supported(layer->d, B, layer->wdtype) && !cats_fused_supported(layer->d, B, layer->wdtype) &&
       (size_t)batch_tier(B) * layer->d * esize(layer->wdtype) > kMaxDynSmem)
     return CSFFN_ERR_UNSUPPORTED_SHAPE;
   return check_ws(ws, ws_bytes, ws_layout(layer->d, layer->h, B, 0).ybuf);
@@ -234,7 +234,8 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   if ((cand_idx == nullptr) != (cand_count == nullptr)) return CSFFN_ERR_INVALID_ARG;
   if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
   if ((st = check_cats_step(layer, x, B, t, idx, a_val, out, ws, ws_bytes)) != CSFFN_OK) return st;
-  if (!cats_fused_supported(layer->d, B, layer->wdtype)) {
+  const bool ring = cats_ring_supported(layer->d, B, layer->wdtype);
+  if (!ring && !cats_fused_supported(layer->d, B, layer->wdtype)) {
     st = csffn_gate_mask(layer, x, B, t, cand_idx, cand_count, idx, count, a_val, ws, ws_bytes, stream);
     if (st != CSFFN_OK) return st;
     return csffn_sparse_ffn_forward(layer, x, B, idx, count, a_val, out, out_mode, ws, ws_bytes, stream);
@@ -264,7 +265,8 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   a.a_val = a_val;
   a.out = out;
   a.out_mode = out_mode;
-  return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
+  return cuda_status(ring ? launch_cats_ring(a, layer->wdtype, as_stream(stream))
+                          : launch_cats_fused(a, layer->wdtype, as_stream(stream)));
 }
 
 csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,

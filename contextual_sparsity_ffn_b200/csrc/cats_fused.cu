@@ -33,6 +33,7 @@
 // is bounded; the counters return to zero by themselves (the ticket counter is cleared by the
 // last CTA to arrive at the meeting).
 #include "common.cuh"
+#include "fused_end.cuh"
 #include "gemv.cuh"
 #include "kernels.h"
 #include "tma.cuh"
@@ -44,52 +45,9 @@ constexpr int kFusedWarps = kFusedThreads / kWarp;
 constexpr int kChunk = kFusedWarps;  // neuron rows per chunk, one per warp
 constexpr int kQueueBatch = kFusedWarps;      // kept rows per up/down batch, one W_up row per warp
 constexpr int kQueueSlots = 2 * kQueueBatch;  // ring of queued kept rows (a chunk adds at most kChunk)
-constexpr int kCounters = 1;         // ticket counters (one: measured faster than 4 or 32 blocks)
-constexpr int kCounterStride = 32;   // 32-bit words between counters (128 bytes)
+constexpr int kCounters = kTicketCounters;
 constexpr int kTailChunk = 4;        // rows per chunk at the end of the row range
 constexpr int kTailGrids = 2;        // the last kTailGrids * grid chunks are of kTailChunk rows
-
-// Fused control words (FusedArgs::ctl).
-constexpr int kCtlDone = 0;  // CTAs whose partial sums and flags are written (wraps to 0 on the last)
-constexpr int kCtlY = 2;     // CTAs whose share of the predictor's y is written (predictor mode)
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// out[0..3] += (a, b, c, e) as one vector reduction in L2 (no return value); 16-byte aligned.
-__device__ __forceinline__ void red_add_v4(float* out, float a, float b, float c, float e) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(a), "f"(b), "f"(c), "f"(e)
-               : "memory");
-}
-
-// Bounded wait until *p == 0 (acquire).  Gives up after a second and records the timeout.
-__device__ __forceinline__ void wait_zero(const uint32_t* p, uint32_t* err) {
-  if (ld_acquire_u32(p) == 0u) return;
-  const uint64_t t0 = globaltimer_now();
-  while (ld_acquire_u32(p) != 0u) {
-    if (globaltimer_now() - t0 > 1000000000ull) {
-      atomicOr(err, kDevErrTimeout);
-      return;
-    }
-    __nanosleep(64);
-  }
-}
-
-// Bounded wait until *p >= target (acquire).  Gives up after a second and records the timeout.
-__device__ __forceinline__ void wait_at_least(const uint32_t* p, uint32_t target, uint32_t* err) {
-  if (ld_acquire_u32(p) >= target) return;
-  const uint64_t t0 = globaltimer_now();
-  while (ld_acquire_u32(p) < target) {
-    if (globaltimer_now() - t0 > 1000000000ull) {
-      atomicOr(err, kDevErrTimeout);
-      return;
-    }
-    __nanosleep(64);
-  }
-}
 
 // acc[b] += W[row] . x_b over this lane's share (U 16-byte vectors in flight per lane).
 template <typename WT, int NB, int U>
@@ -208,13 +166,6 @@ __device__ __forceinline__ void smem_row_dot(const WT* row, const WT* xs, int K,
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void named_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-constexpr int kHalf = kFusedThreads / 2;  // threads of each end-phase group
-constexpr int kCountLoads = 16;           // 16-byte flag loads in flight per thread (compaction)
-
 // acc[b] += row[0 .. n) . y_b[0 .. n): a row in shared memory against fp32 vectors y_b = ys + b * n.
 template <typename WT, int NB>
 __device__ __forceinline__ void smem_dot_f32(const WT* row, const float* ys, int n, int lane, float (&acc)[NB]) {
@@ -476,7 +427,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
   int kr = 0;  // predictor mode: rounds so far (parity of their keep flags)
   for (int it = 0; chunk >= 0; ++it) {
     const int buf = it & 1;
-    mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort);
+    // A copy that never lands (a wait that ran out: the error word is set) ends the chunk loop in
+    // every thread together, so no math runs on a buffer that did not arrive.
+    if (__syncthreads_or(!mbar_wait(&s_bar, (uint32_t)(it & 1), p.err, &s_abort))) break;
     int j0, n_in;
     cm.rows(chunk, j0, n_in);
     int next;
@@ -595,131 +548,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) cats_fused_kernel(const Fuse
       }
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    // The arrival counter wraps back to zero on the last arrival (atomicInc); the others wait for
-    // that zero (their own arrival keeps it above zero until then), so it is ready for the next
-    // launch without a reset.  Every CTA has drawn its last ticket (and passed the predictor's
-    // count) before it arrives, so the last one also clears those counters for the next launch.
-    if (atomicInc(&p.ctl[kCtlDone], gridDim.x - 1u) == gridDim.x - 1u) {
-      for (int i = 0; i < kCounters; ++i) {
-        p.tickets[i * kCounterStride] = 0u;
-        p.tickets[i * kCounterStride + 1] = 0u;
-      }
-      p.ctl[kCtlY] = 0u;
-      __threadfence();  // with the counter read above: the other CTAs' sums are visible here
-    } else {
-      wait_zero(&p.ctl[kCtlDone], p.err);
-    }
-  }
-  __syncthreads();
-
-  if (warp < kHalf / kWarp) {
-    // ------------------------------------------------------------ out = the accumulators' sum
-    // CTA k takes an equal share of the B*d/4 float4 columns, writes their sum (plus the old out
-    // when accumulating) and clears them for the next launch.
-    const int n4 = B * d / 4;
-    const int i0 = (int)((long long)n4 * blockIdx.x / gridDim.x);
-    const int i1 = (int)((long long)n4 * (blockIdx.x + 1) / gridDim.x);
-    for (int i = i0 + tid; i < i1; i += kHalf) {
-      float4 s4[kFusedAccCopies];
-#pragma unroll
-      for (int c = 0; c < kFusedAccCopies; ++c)
-        s4[c] = __ldcg(reinterpret_cast<const float4*>(p.facc + (size_t)c * B * d) + i);
-      float4 t4 = s4[0];
-#pragma unroll
-      for (int c = 1; c < kFusedAccCopies; ++c) {
-        t4.x += s4[c].x;
-        t4.y += s4[c].y;
-        t4.z += s4[c].z;
-        t4.w += s4[c].w;
-      }
-      if (p.out_mode == CSFFN_OUT_BF16) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(t4.x, t4.y), hi = __floats2bfloat162_rn(t4.z, t4.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(p.out)[i] = pk;
-      } else {
-        float4* of = reinterpret_cast<float4*>(p.out) + i;
-        if (p.out_mode == CSFFN_OUT_F32_ACCUMULATE) {
-          const float4 prev = *of;
-          t4.x += prev.x;
-          t4.y += prev.y;
-          t4.z += prev.z;
-          t4.w += prev.w;
-        }
-        *of = t4;
-      }
-#pragma unroll
-      for (int c = 0; c < kFusedAccCopies; ++c)
-        __stcg(reinterpret_cast<float4*>(p.facc + (size_t)c * B * d) + i, make_float4(0.f, 0.f, 0.f, 0.f));
-    }
-  } else {
-    // ------------------------------------------------------------ compaction of the active list
-    // CTA k owns the 32-position words [wa, wb); the kept positions before wa are counted from the
-    // flag bytes (each 0 or 1, so the popcount of a 32-bit word of flags counts its kept rows).
-    // Position j is written out as its neuron (ascending, as the candidate list is).  The flags and
-    // activations of the first pass are loaded before that count, so the two round trips overlap.
-    const int ct = tid - kHalf, cw = warp - kHalf / kWarp;
-    const int n_words = (n_rows + kWarp - 1) / kWarp;
-    const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
-    const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
-    if (wa < wb || blockIdx.x == gridDim.x - 1) {
-      bool f;
-      int nr;
-      float av[NB];
-      auto load_pass = [&](int w0) {  // flag, neuron and activations of position (w0 + cw) * 32 + lane
-        const int jp = (w0 + cw) * kWarp + lane;
-        const bool in = w0 + cw < wb && jp < n_rows;
-        f = in && __ldcg(p.flags + jp) != 0;
-        nr = in ? neuron(jp) : 0;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
-      };
-      load_pass(wa);
-      uint32_t before = 0;
-      const uint4* f4 = reinterpret_cast<const uint4*>(p.flags);
-      for (int i0 = ct; i0 < wa * 2; i0 += kHalf * kCountLoads) {  // each batch's loads issued together
-        uint4 fw[kCountLoads];
-#pragma unroll
-        for (int u = 0; u < kCountLoads; ++u)
-          fw[u] = i0 + u * kHalf < wa * 2 ? __ldcg(f4 + i0 + u * kHalf) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int u = 0; u < kCountLoads; ++u) before += __popc(fw[u].x) + __popc(fw[u].y) + __popc(fw[u].z) + __popc(fw[u].w);
-      }
-      before = warp_sum_u32(before);
-      if (lane == 0) s_cnt[cw] = before;
-      named_sync(2, kHalf);
-      uint32_t base = 0;
-#pragma unroll
-      for (int w = 0; w < kHalf / kWarp; ++w) base += s_cnt[w];
-      named_sync(2, kHalf);
-      for (int w0 = wa; w0 < wb; w0 += kHalf / kWarp) {
-        const uint32_t m = __ballot_sync(0xffffffffu, f);
-        if (lane == 0) s_cnt[cw] = __popc(m);
-        named_sync(2, kHalf);
-        uint32_t off = base, total = base;
-#pragma unroll
-        for (int ww = 0; ww < kHalf / kWarp; ++ww) {
-          off += ww < cw ? s_cnt[ww] : 0u;
-          total += s_cnt[ww];
-        }
-        if (f) {
-          const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
-          p.idx[pos] = nr;
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-            if (b < B) p.a_val[(size_t)b * h + pos] = av[b];
-        }
-        base = total;
-        named_sync(2, kHalf);
-        load_pass(w0 + kHalf / kWarp);
-      }
-      if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
-    }
-  }
+  fused_finish<NB>(p, n_rows, s_cnt);
 }
 
 // Dynamic shared memory: the staged tokens and one chunk of prefetched rows (W_gate, or V_r in

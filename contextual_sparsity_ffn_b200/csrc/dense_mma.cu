@@ -13,8 +13,9 @@
 // chunks) are read with the same permutation of k.  Epilogue: v[b, i] = act(z + beta) * u.
 //
 // Down (down_mma_kernel): out[b, :] = sum_i v[b, i] W_down^T[i, :] with M = tokens, N = output
-// columns and K = neurons.  W_down^T rows and the matching slice of v are staged in shared memory
-// (cp.async, four-block ring, padded rows); W_down^T is read as B fragments by ldmatrix .trans.
+// columns and K = neurons.  Tiles of W_down^T (64 neurons x 64 columns) and the matching tiles of v
+// arrive by TMA tensor copies (cp.async.bulk.tensor with the 128-byte swizzle, no multicast) in a
+// four-stage ring on mbarriers; W_down^T is read as B fragments by ldmatrix .trans.
 // The gate/up epilogue stores v as bf16 high and low parts (two MMAs), so
 // the product carries about 16 mantissa bits of v.  Column tiles x neuron ranges, partials
 // summed by the last CTA of each column tile (in range order).

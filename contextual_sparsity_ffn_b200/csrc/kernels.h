@@ -139,6 +139,10 @@ struct FusedArgs {
 };
 bool cats_fused_supported(int d, int B, int wdtype, int rank = 0);
 cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
+// The same step (CATS or candidate mode, not the predictor mode) on a shared-memory ring fed by
+// bulk copies from one producer warp (ring.cu): one CTA per SM.
+bool cats_ring_supported(int d, int B, int wdtype);
+cudaError_t launch_cats_ring(const FusedArgs& a, int wdtype, cudaStream_t s);
 
 // Radix selection and per-neuron selection (calibration).
 size_t kth_state_bytes();

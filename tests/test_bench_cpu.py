@@ -1,4 +1,5 @@
 """Host logic of bench.py that needs no GPU: the profiled-traffic gate and the whole-job arithmetic."""
+import json
 import os
 import sys
 
@@ -10,15 +11,17 @@ import bench  # noqa: E402
 
 
 def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
-    summary = tmp_path / "profile.md"
-    summary.write_text(f"traffic_bytes_per_launch: 183014144\ncsrc_sha256_16: {bench.csrc_hash()}\n")
-    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(summary))
+    rec = tmp_path / "profile.json"
+    monkeypatch.setattr(bench, "PROFILE_JSON", str(rec))
+    rec.write_text(json.dumps({"traffic_bytes_per_launch": 183014144, "csrc_sha256_16": bench.csrc_hash()}))
     assert bench.profiled_traffic() == 183014144.0
-    summary.write_text("traffic_bytes_per_launch: 183014144\ncsrc_sha256_16: 0000000000000000\n")
+    rec.write_text(json.dumps({"traffic_bytes_per_launch": 183014144, "csrc_sha256_16": "0000000000000000"}))
     assert bench.profiled_traffic() is None  # the kernel source changed since the capture
-    summary.write_text(f"csrc_sha256_16: {bench.csrc_hash()}\n")
+    rec.write_text(json.dumps({"csrc_sha256_16": bench.csrc_hash()}))
     assert bench.profiled_traffic() is None  # no traffic figure
-    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(tmp_path / "missing.md"))
+    rec.write_text("not json")
+    assert bench.profiled_traffic() is None
+    monkeypatch.setattr(bench, "PROFILE_JSON", str(tmp_path / "missing.json"))
     assert bench.profiled_traffic() is None
 
 
