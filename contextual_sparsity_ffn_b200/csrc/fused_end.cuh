@@ -1,10 +1,9 @@
-// End phase shared by the one-launch decode kernels: one grid-wide meeting, then the output (the
-// sum of the CTAs' partial outputs in L2) and the compaction of the active list.
+// End phase shared by the decode-step kernels: the output (the sum of the CTAs' partial outputs in
+// L2) and the compaction of the active list.
 //
-// Before calling fused_finish every CTA has added its partial output into one of
-// kFusedAccCopies fp32 accumulators in the workspace (red_add_v4) and written the keep flag and the
-// kept activations of every row position it decided.  The kernels run as cooperative launches, so
-// all CTAs are co-resident and the meeting cannot wait on a CTA that has not started.
+// Before it every CTA of the step has added its partial output into one of kFusedAccCopies fp32
+// accumulators in the workspace (red_add_v4) and written the keep flag and the kept activations of
+// every row position it decided.
 #pragma once
 
 #include "common.cuh"
@@ -72,36 +71,18 @@ __device__ __forceinline__ int step_neuron(const int32_t* cand, int h, int j) {
   return (unsigned)r < (unsigned)h ? r : 0;
 }
 
-// The meeting and the end phase, called by every thread of the CTA (blockDim.x >= 2 * kFinishHalf)
-// after its partial output is in the accumulators.  Threads [0, kFinishHalf) write out (the sum of
+// The end phase, called by every thread of the CTA (blockDim.x >= 2 * kFinishHalf) once every CTA's
+// partial output is in the accumulators and every keep flag is written (after the meeting below, or
+// in a kernel that follows the one that wrote them).  Threads [0, kFinishHalf) write out (the sum of
 // the accumulators, plus the old out when accumulating) over an equal share of the columns and
 // clear the accumulators for the next launch; threads [kFinishHalf, 2 kFinishHalf) compact idx /
 // a_val / count from the keep flags: CTA k owns a fixed range of 32-position words, counts the kept
 // positions before it from the flag bytes (each 0 or 1, so a 32-bit word's popcount counts its
-// kept rows) and writes its positions' neurons in ascending order.  The arrival counter wraps to
-// zero on the last arrival (atomicInc) and the others wait for that zero, so it is ready for the
-// next launch without a reset; the last CTA also clears the ticket counter and the predictor's
-// count (every CTA has drawn its last ticket and passed that count before it arrives).
+// kept rows) and writes its positions' neurons in ascending order.
 template <int NB>
-__device__ void fused_finish(const FusedArgs& p, int n_rows, uint32_t* s_cnt) {
+__device__ void fused_finish_work(const FusedArgs& p, int n_rows, uint32_t* s_cnt) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = p.B, d = p.d, h = p.h;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    if (atomicInc(&p.ctl[kCtlDone], gridDim.x - 1u) == gridDim.x - 1u) {
-      for (int i = 0; i < kTicketCounters; ++i) {
-        p.tickets[i * kCounterStride] = 0u;
-        p.tickets[i * kCounterStride + 1] = 0u;
-      }
-      p.ctl[kCtlY] = 0u;
-      __threadfence();  // with the counter read above: the other CTAs' sums are visible here
-    } else {
-      wait_zero(&p.ctl[kCtlDone], p.err);
-    }
-  }
-  __syncthreads();
-
   if (tid < kFinishHalf) {
     const int n4 = B * d / 4;
     const int i0 = (int)((long long)n4 * blockIdx.x / gridDim.x);
@@ -200,6 +181,31 @@ __device__ void fused_finish(const FusedArgs& p, int n_rows, uint32_t* s_cnt) {
       if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
     }
   }
+}
+
+// One grid-wide meeting, then the end phase.  The arrival counter wraps to zero on the last arrival
+// (atomicInc) and the others wait for that zero, so it is ready for the next launch without a
+// reset; the last CTA also clears the ticket counter and the predictor's count (every CTA has drawn
+// its last ticket and passed that count before it arrives).  Only for cooperative launches: all
+// CTAs are co-resident, so the meeting cannot wait on a CTA that has not started.
+template <int NB>
+__device__ void fused_finish(const FusedArgs& p, int n_rows, uint32_t* s_cnt) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (atomicInc(&p.ctl[kCtlDone], gridDim.x - 1u) == gridDim.x - 1u) {
+      for (int i = 0; i < kTicketCounters; ++i) {
+        p.tickets[i * kCounterStride] = 0u;
+        p.tickets[i * kCounterStride + 1] = 0u;
+      }
+      p.ctl[kCtlY] = 0u;
+      __threadfence();  // with the counter read above: the other CTAs' sums are visible here
+    } else {
+      wait_zero(&p.ctl[kCtlDone], p.err);
+    }
+  }
+  __syncthreads();
+  fused_finish_work<NB>(p, n_rows, s_cnt);
 }
 
 }  // namespace csffn

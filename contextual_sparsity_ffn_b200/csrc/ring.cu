@@ -1,6 +1,6 @@
-// One-launch CATS decode step on shared-memory rings fed by bulk copies: gate, threshold, up and
-// down projection of one FFN layer, then one grid meeting, the output and the compaction of the
-// active list.
+// CATS decode step on shared-memory rings fed by bulk copies: gate, threshold, up and down
+// projection of one FFN layer in one streaming kernel, then the output and the compaction of the
+// active list in a short second kernel.
 //
 // "CATS: Contextually-Aware Thresholding for Sparsity in Large Language Models", abstract and the
 // section on the custom kernel: the gate GEMV, the compare against t, and the flag-gated up and down
@@ -8,8 +8,7 @@
 // neurons that survive the threshold.  A decode step moves 100-300 MB, so it is bound by how many
 // bytes each SM keeps in flight, and by the dependent round trip gate -> up -> down at the end.
 //
-// One CTA per SM (a cooperative launch, so the grid meeting at the end cannot wait on a CTA that
-// has not started).  Every weight row reaches shared memory by one 1-D bulk copy (cp.async.bulk, no
+// One CTA per SM.  Every weight row reaches shared memory by one 1-D bulk copy (cp.async.bulk, no
 // tensor map, no multicast), completing on its slot's mbarrier.  Warps:
 //   1 .. 8   gate warps.  Each is its own stream: it draws tickets of kRingChunk gate rows from one
 //            counter (its first chunk is fixed), keeps R rows in flight in its own R slots, dots each
@@ -22,6 +21,13 @@
 //            for them in registers; a slot of the down ring is released when all eight are done.
 // No warp handles a row it does no work on, and the gate path has no central issuer: the bytes in
 // flight are the gate warps' slots (16 rows per SM at d = 4096) plus the down ring.
+// No CTA waits for another: each adds its partial output into the workspace accumulators, writes
+// the keep flags of its rows and exits; a small second kernel (ring_finish_kernel) writes out and
+// compacts idx / a_val / count.  Both are launched as programmatic dependents of the kernel before
+// them on the stream: a streaming CTA may start on an SM the previous step's streaming CTA has left
+// while the previous step still finishes, and it fetches its first W_gate rows (weights, which no
+// kernel writes) before griddepcontrol.wait; everything else -- the tokens, the candidate list, the
+// workspace, the outputs -- is touched only after it.
 // Every wait is bounded (a second); a wait that runs out records the timeout in the error word and
 // ends the CTA's loops, after waiting (again bounded) for the CTA's own copies still in flight.
 #include "common.cuh"
@@ -144,11 +150,13 @@ struct RingShared {
   int abort;
 };
 
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <typename WT, int NB, int KV>
 __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedArgs p, const RingGeom geo) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ RingShared sh;
-  __shared__ uint32_t s_cnt[kFinishHalf / kWarp];
   constexpr int EPV = Vec<WT>::N;
   constexpr int XH = EPV / 4;  // float4 halves of a 16-byte weight vector
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -172,9 +180,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
   volatile int* dq_flag = reinterpret_cast<volatile int*>(smem_raw + L.dq_flag);
   volatile int* abort = &sh.abort;
 
+  pdl_launch_dependents();  // the next step may start on the SMs this one leaves
+
+  // A candidate list (and its count) may come from the kernel before: read after the wait.
   const int32_t* cand = p.cand_idx;
-  const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
-  const int n_chunks = (n_rows + kRingChunk - 1) / kRingChunk;
   const int n_streams = (int)gridDim.x * kGateWarps;  // gate warps in the grid; chunk g goes to stream g first
 
   if (tid == 0) {
@@ -194,6 +203,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
 
   if (warp == 0) {
     // ------------------------------------------------------------------------------ producer
+    pdl_wait();
     const WT* Wd = reinterpret_cast<const WT*>(p.W_down_t);
     int head = 0, dseq = 0, ddone = 0;
     bool ok = true;
@@ -284,6 +294,40 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     uint64_t* full = gfull + (gw << LR);
     RingDesc* desc = gdesc + (gw << LR);
     WT* ring = gring + ((size_t)gw << LR) * d;
+    const int stream = (int)blockIdx.x * kGateWarps + gw;
+    const float zero[NB] = {};
+
+    // lane 0 fills the slot's descriptor and issues its row (the slot's previous row was read by
+    // this warp, whose lanes finished with it before the warp barrier that precedes every issue)
+    auto issue = [&](int q, int kind, int j, int n, float beta, const float (&a)[NB], const WT* src) {
+      const int s = q & (R - 1);
+      if (lane == 0) {
+        RingDesc& ds = desc[s];
+        ds.kind = kind;
+        ds.j = j;
+        ds.n = n;
+        ds.beta = beta;
+#pragma unroll
+        for (int b = 0; b < kFusedMaxBatch; ++b) ds.a[b] = b < NB ? a[b] : 0.f;
+        mbar_arrive_expect_tx(&full[s], rowbytes);
+        bulk_load(ring + (size_t)s * d, src, rowbytes, &full[s]);
+      }
+    };
+    // Without a candidate list the stream's first chunk is rows 2 stream and 2 stream + 1 of W_gate:
+    // its copies go out before the wait (and before the tokens are staged).
+    int iss = 0;  // items issued; item q sits in slot q mod R
+    int pre = 0;  // rows of the first chunk issued before the wait
+    if (!cand && stream * kRingChunk < h) {
+      const int rows = min(kRingChunk, min(R, h - stream * kRingChunk));
+      for (int i = 0; i < rows; ++i) {
+        const int n = stream * kRingChunk + i;
+        issue(iss++, kItemGate, n, n, p.bias ? __ldg(p.bias + n) : 0.f, zero, Wg + (size_t)n * d);
+      }
+      pre = rows;
+    }
+    pdl_wait();
+    const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
+    const int n_chunks = (n_rows + kRingChunk - 1) / kRingChunk;
     // tokens -> shared memory as fp32 (zero past B), then a barrier among the gate warps
     for (int e = tid - kWarp; e < NB * NV; e += kGateWarps * kWarp) {
       const int b = e / NV, v = e - b * NV;
@@ -300,7 +344,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     // Chunks of gate rows: this stream's first chunk is its own number; later ones come from the
     // ticket counter (a draw one chunk ahead of its use).  Lane i < kRingChunk holds the neuron and
     // the gate bias of row i of a resolved chunk.
-    const int stream = (int)blockIdx.x * kGateWarps + gw;
     uint32_t ticket = 0;  // lane 0: a draw in flight
     bool drawn = false;
     if (lane == 0 && n_streams < n_chunks) ticket = atomicAdd(p.tickets, 1u);
@@ -327,7 +370,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
       n = in ? step_neuron(cand, h, j) : 0;
       beta = (in && p.bias) ? __ldg(p.bias + n) : 0.f;
     };
-    int cur_c = stream < n_chunks ? next_chunk() : (first = -1, -1), cur_i = 0, cur_n, nxt_n;
+    int cur_c = stream < n_chunks ? next_chunk() : (first = -1, -1), cur_i = pre, cur_n, nxt_n;
     float cur_b, nxt_b;
     chunk_row(cur_c, cur_n, cur_b);
     int nxt_c = cur_c >= 0 ? next_chunk() : -1;
@@ -345,23 +388,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
       return true;
     };
 
-    // lane 0 fills the slot's descriptor and issues its row (the slot's previous row was read by
-    // this warp, whose lanes finished with it before the warp barrier that precedes every issue)
-    auto issue = [&](int q, int kind, int j, int n, float beta, const float (&a)[NB], const WT* src) {
-      const int s = q & (R - 1);
-      if (lane == 0) {
-        RingDesc& ds = desc[s];
-        ds.kind = kind;
-        ds.j = j;
-        ds.n = n;
-        ds.beta = beta;
-#pragma unroll
-        for (int b = 0; b < kFusedMaxBatch; ++b) ds.a[b] = b < NB ? a[b] : 0.f;
-        mbar_arrive_expect_tx(&full[s], rowbytes);
-        bulk_load(ring + (size_t)s * d, src, rowbytes, &full[s]);
-      }
-    };
-    const float zero[NB] = {};
     auto issue_gate_row = [&](int q) {
       const int n = __shfl_sync(kFullMask, cur_n, cur_i);
       const float beta = __shfl_sync(kFullMask, cur_b, cur_i);
@@ -369,7 +395,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
       ++cur_i;
     };
 
-    int iss = 0;  // items issued; item q sits in slot q mod R
     while (iss < R && gate_row_left()) issue_gate_row(iss++);
     bool ok = true;
     for (int k = 0; k < iss; ++k) {
@@ -483,6 +508,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
   } else {
     // ------------------------------------------------------------------------------ down warps
     // Down warp cw owns the 16-byte column vectors cw*32 + lane + k*256 (k < KV) of out.
+    pdl_wait();
     const int cw = warp - 1 - kGateWarps;
     float acc[NB][KV][EPV];
 #pragma unroll
@@ -532,7 +558,24 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
       }
     }
   }
-  fused_finish<NB>(p, n_rows, s_cnt);
+}
+
+// The end of the step, in a kernel of its own after the streaming kernel (the kernel boundary is the
+// grid-wide barrier): the output and the compaction of idx / a_val / count, spread over the grid;
+// CTA 0 clears the ticket counter for the next step.  Launched as a programmatic dependent too: its
+// CTAs may start beside the streaming kernel's and wait there, and the next step's streaming kernel
+// may start beside them.
+template <int NB>
+__global__ void __launch_bounds__(2 * kFinishHalf) ring_finish_kernel(const FusedArgs p) {
+  __shared__ uint32_t s_cnt[kFinishHalf / kWarp];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int n_rows = p.cand_idx ? min(max(__ldg(p.cand_count), 0), p.h) : p.h;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.tickets[0] = 0u;
+    p.tickets[1] = 0u;
+  }
+  fused_finish_work<NB>(p, n_rows, s_cnt);
 }
 
 // 16-byte vectors per lane of the down projection's columns for a shape (0 when the ring kernel does
@@ -558,7 +601,7 @@ static cudaError_t ring_t(const FusedArgs& a, cudaStream_t st) {
   const RingGeom geo = ring_geom(a.d, (int)sizeof(WT), NB);
   if (geo.lr < 0) return cudaErrorInvalidValue;
   const size_t smem = ring_smem(a.d, (int)sizeof(WT), NB, geo).total;
-  // The shared-memory attribute and the co-residency check, once per device and instance (again
+  // The shared-memory attribute and the one-CTA-per-SM check, once per device and instance (again
   // when a larger shape needs more shared memory).
   static int ready[64] = {0};
   int dev = 0;
@@ -574,17 +617,22 @@ static cudaError_t ring_t(const FusedArgs& a, cudaStream_t st) {
     if (occ < 1) return cudaErrorInvalidConfiguration;
     ready[dev] = (int)smem;
   }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sm_count());
   cfg.blockDim = dim3(kRingThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, geo);
+  e = cudaLaunchKernelEx(&cfg, kern, a, geo);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t fin = cfg;
+  fin.blockDim = dim3(2 * kFinishHalf);
+  fin.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&fin, ring_finish_kernel<NB>, a);
 }
 
 template <typename WT, int NB>
