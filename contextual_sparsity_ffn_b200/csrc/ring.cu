@@ -42,6 +42,7 @@ constexpr int kDownWarps = 8;
 constexpr int kRingThreads = (1 + kGateWarps + kDownWarps) * kWarp;
 constexpr int kRingChunk = 2;      // gate rows per ticket
 constexpr int kDownQueue = 64;     // kept neurons between the gate warps and the producer
+constexpr bool kPrefetchBeforeWait = true;
 constexpr size_t kRingSmemBudget = 220 * 1024;
 constexpr uint32_t kFullMask = 0xffffffffu;
 
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
           // the down warps released this slot (arrive, release) after their reads of its previous
           // row, and this lane acquired that: the copy may overwrite it
           mbar_arrive_expect_tx(&dfull[sd], rowbytes);
-          bulk_load(dring + (size_t)sd * d, Wd + (size_t)e.n * d, rowbytes, &dfull[sd]);
+          bulk_load_hint(dring + (size_t)sd * d, Wd + (size_t)e.n * d, rowbytes, &dfull[sd], l2_evict_first_policy());
         }
         __syncwarp();
         head += m;
@@ -310,14 +311,14 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
 #pragma unroll
         for (int b = 0; b < kFusedMaxBatch; ++b) ds.a[b] = b < NB ? a[b] : 0.f;
         mbar_arrive_expect_tx(&full[s], rowbytes);
-        bulk_load(ring + (size_t)s * d, src, rowbytes, &full[s]);
+        bulk_load_hint(ring + (size_t)s * d, src, rowbytes, &full[s], l2_evict_first_policy());
       }
     };
     // Without a candidate list the stream's first chunk is rows 2 stream and 2 stream + 1 of W_gate:
     // its copies go out before the wait (and before the tokens are staged).
     int iss = 0;  // items issued; item q sits in slot q mod R
     int pre = 0;  // rows of the first chunk issued before the wait
-    if (!cand && stream * kRingChunk < h) {
+    if (kPrefetchBeforeWait && !cand && stream * kRingChunk < h) {
       const int rows = min(kRingChunk, min(R, h - stream * kRingChunk));
       for (int i = 0; i < rows; ++i) {
         const int n = stream * kRingChunk + i;
@@ -328,6 +329,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     pdl_wait();
     const int n_rows = cand ? min(max(__ldg(p.cand_count), 0), h) : h;
     const int n_chunks = (n_rows + kRingChunk - 1) / kRingChunk;
+    // The first ticket draw goes out now, so that its round trip overlaps the staging of the tokens.
+    uint32_t ticket = 0;  // lane 0: a draw in flight
+    if (lane == 0 && n_streams < n_chunks) ticket = atomicAdd(p.tickets, 1u);
+    bool drawn = n_streams < n_chunks;
     // tokens -> shared memory as fp32 (zero past B), then a barrier among the gate warps
     for (int e = tid - kWarp; e < NB * NV; e += kGateWarps * kWarp) {
       const int b = e / NV, v = e - b * NV;
@@ -344,10 +349,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     // Chunks of gate rows: this stream's first chunk is its own number; later ones come from the
     // ticket counter (a draw one chunk ahead of its use).  Lane i < kRingChunk holds the neuron and
     // the gate bias of row i of a resolved chunk.
-    uint32_t ticket = 0;  // lane 0: a draw in flight
-    bool drawn = false;
-    if (lane == 0 && n_streams < n_chunks) ticket = atomicAdd(p.tickets, 1u);
-    drawn = n_streams < n_chunks;
     int first = stream < n_chunks ? stream : -1;
     auto next_chunk = [&]() -> int {
       if (first >= 0) {
@@ -466,8 +467,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
           for (int b = 0; b < NB; ++b)
             if (b < B) p.afull[(size_t)b * h + ds.j] = a[b];
         }
-        if (kept)  // the freed slot takes the neuron's W_up row
+        if (kept) {
+          // The freed slot takes the neuron's W_up row; its W_down^T row, which the producer copies
+          // once the up dot is done, is fetched into L2 now, so that copy does not wait on HBM.
+          if (lane == 0) bulk_prefetch_l2(reinterpret_cast<const WT*>(p.W_down_t) + (size_t)ds.n * d, rowbytes);
           issue(iss++, kItemUp, 0, ds.n, 0.f, a, Wu + (size_t)ds.n * d);
+        }
         else if (gate_row_left())
           issue_gate_row(iss++);
       } else {
