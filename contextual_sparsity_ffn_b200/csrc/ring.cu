@@ -347,45 +347,47 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     named_sync(1, kGateWarps * kWarp);
 
     // Chunks of gate rows: this stream's first chunk is its own number; later ones come from the
-    // ticket counter (a draw one chunk ahead of its use).  Lane i < kRingChunk holds the neuron and
-    // the gate bias of row i of a resolved chunk.
-    int first = stream < n_chunks ? stream : -1;
-    auto next_chunk = [&]() -> int {
-      if (first >= 0) {
-        const int c = first;
-        first = -1;
-        return c;
-      }
-      if (!drawn) return -1;
-      const int c = n_streams + (int)__shfl_sync(kFullMask, ticket, 0);
-      if (c >= n_chunks) {
-        drawn = false;
-        return -1;
-      }
-      if (lane == 0) ticket = atomicAdd(p.tickets, 1u);
-      return c;
-    };
+    // ticket counter.  A ticket is drawn when the current chunk's last row goes out (the first one
+    // right after the wait), so its round trip hides behind the row in flight, and when the counter
+    // runs dry a warp holds no more than the rows of its current chunk and one drawn chunk.  Lane
+    // i < kRingChunk holds the neuron and the gate bias of row i of the current chunk.
+    auto chunk_rows = [&](int c) { return min(kRingChunk, n_rows - c * kRingChunk); };
     auto chunk_row = [&](int c, int& n, float& beta) {
       const int j = c * kRingChunk + lane;
       const bool in = c >= 0 && lane < kRingChunk && j < n_rows;
       n = in ? step_neuron(cand, h, j) : 0;
       beta = (in && p.bias) ? __ldg(p.bias + n) : 0.f;
     };
-    int cur_c = stream < n_chunks ? next_chunk() : (first = -1, -1), cur_i = pre, cur_n, nxt_n;
-    float cur_b, nxt_b;
+    bool more = n_streams < n_chunks;  // the counter may still hand out chunks
+    int cur_c = stream < n_chunks ? stream : -1, cur_i = pre, cur_n;
+    float cur_b;
     chunk_row(cur_c, cur_n, cur_b);
-    int nxt_c = cur_c >= 0 ? next_chunk() : -1;
-    chunk_row(nxt_c, nxt_n, nxt_b);
+    auto draw = [&]() {
+      if (lane == 0) ticket = atomicAdd(p.tickets, 1u);
+      drawn = true;
+    };
     auto gate_row_left = [&]() -> bool {  // moves to the next chunk when the current one is issued
       if (cur_c < 0) return false;
-      if (cur_i < min(kRingChunk, n_rows - cur_c * kRingChunk)) return true;
-      cur_c = nxt_c;
-      cur_n = nxt_n;
-      cur_b = nxt_b;
+      const int rows = chunk_rows(cur_c);
+      if (cur_i < rows) {
+        if (cur_i == rows - 1 && more && !drawn) draw();
+        return true;
+      }
+      if (!more) {
+        cur_c = -1;
+        return false;
+      }
+      if (!drawn) draw();
+      const int c = n_streams + (int)__shfl_sync(kFullMask, ticket, 0);
+      drawn = false;
+      if (c >= n_chunks) {
+        more = false;
+        cur_c = -1;
+        return false;
+      }
+      cur_c = c;
       cur_i = 0;
-      if (cur_c < 0) return false;
-      nxt_c = next_chunk();
-      chunk_row(nxt_c, nxt_n, nxt_b);
+      chunk_row(cur_c, cur_n, cur_b);
       return true;
     };
 
