@@ -6,16 +6,16 @@ accumulation, batch-1 decode, CATS threshold calibrated by csffn_calibrate_thres
 on 512 seeded calibration vectors at 50% target sparsity (70% and 90% and the dense
 path of the same library are measured too and reported under "detail").
 
-A step is one CATS decode of one layer through csffn_cats_ffn_forward: gate GEMV + SiLU
-+ threshold, the gathered up and down projections of the kept rows, then one grid meeting,
-the sum of the CTAs' partial outputs and the compaction of the active list, in one kernel
-launch.  The two-call path
-(csffn_gate_mask then csffn_sparse_ffn_forward, three kernels) is reported under "detail".  The
-timed steps rotate over 8 distinct layer weight sets (2.2 GB, many times the 126 MB L2)
+A step is one CATS decode of one layer through csffn_cats_ffn_forward: gate GEMV + SiLU +
+threshold and the gathered up and down projections of the kept rows in a streaming kernel
+(cats_ring_kernel), then the sum of the CTAs' partial outputs and the compaction of the active list
+in a short finishing kernel (ring_finish_kernel) launched as its programmatic dependent: two
+launches per step.  The two-call path (csffn_gate_mask then csffn_sparse_ffn_forward, three
+kernels) is reported under "detail", with 70% and 90%, the dense path, the SVD-predictor ReGLU
+step, the 32-layer LLaMA-3-8B-shaped stack at batch 1/4/16 and the LLaMA-3-70B-shaped Sirius round.
+The timed steps rotate over 8 distinct layer weight sets (2.2 GB, many times the 126 MB L2)
 so no step reads weights that an earlier step left in L2.  K steps are captured in one
 CUDA graph and timed with CUDA events on the capture stream.
-
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csffn|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica (the decode step has no
 exchange step); the time is the max over ranks and ``value`` is the whole-job time
@@ -263,6 +263,140 @@ def dense_verify_measure(torch, cs, stream, K, W, world, dev):
             f"frac_of_{measured_hbm_gbs()[1]}_hbm": round(nbytes / (us_call * 1e-6) / 1e9 / measured_hbm_gbs()[0], 4)}
 
 
+def device_layer(torch, cs, d, h, gen, dev):
+    """A bf16 SwiGLU layer drawn on the device from a seeded generator, N(0, 0.02^2) (timing only)."""
+    w = [(torch.randn(h, d, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for _ in range(3)]
+    return cs.FFNLayer(w[0], w[1], w[2], cs._abi.ACT_SILU)
+
+
+def time_graph_once(torch, g, stream, warm=2):
+    """One timed replay of a captured graph after `warm` untimed ones (ms)."""
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def stack_measure(torch, cs, stream, world, dev, n_steps=4):
+    """32-layer LLaMA-3-8B-shaped FFN stack (d 4096, h 14336, bf16; 11.3 GB of weights, so every
+    step streams from HBM): per layer xn = bf16(RMSNorm(h)) then h += FFN(xn) in place.  Thresholds
+    per layer at 50% from 512 calibration vectors carried through the dense stack on the device
+    (stack.calibrate_stack).  One step = the 32 layers for B tokens; the residual is reset from the
+    same tokens before each step (inside the graph).  The dense stack is timed the same way."""
+    from contextual_sparsity_ffn_b200 import stack
+    d, h, L = 4096, 14336, 32
+    gen = torch.Generator(device=dev).manual_seed(3)
+    layers = [device_layer(torch, cs, d, h, gen, dev) for _ in range(L)]
+    h_cal = torch.randn(512, d, generator=gen, device=dev)
+    ws16 = cs.new_workspace(layers[0], 16)
+    ts = stack.calibrate_stack(layers, h_cal, 0.5, ws16)
+    h0 = torch.randn(16, d, generator=gen, device=dev)
+    res = {"path": "per layer csffn_rmsnorm_bf16 + csffn_cats_ffn_forward (accumulate; batch 1 and 4 run as "
+                   "the two-kernel step, batch 16 as the gate mask then the gathered up/down); the dense "
+                   "stack: csffn_rmsnorm_bf16 + csffn_dense_ffn_forward", "layers": L, "target_sparsity": 0.5}
+    for B in (1, 4, 16):
+        sb = stack.stack_buffers(layers[0], B)
+        hb = torch.empty(B, d, device=dev)
+        counts = []
+        hb.copy_(h0[:B])
+        stack.sparse_stack(layers, ts, hb, sb, counts=counts)
+
+        def sparse_step(k):
+            hb.copy_(h0[:B])
+            stack.sparse_stack(layers, ts, hb, sb)
+
+        def dense_step(k):
+            hb.copy_(h0[:B])
+            stack.dense_stack(layers, hb, sb.xn, ws16)
+
+        g = run_graph_steps(torch, sparse_step, n_steps, 3, stream)
+        t_sp = max_over_ranks(time_graph_once(torch, g, stream), world, dev) / n_steps
+        del g
+        g = run_graph_steps(torch, dense_step, n_steps, 3, stream)
+        t_de = max_over_ranks(time_graph_once(torch, g, stream), world, dev) / n_steps
+        del g
+        assert cs.check_status(sb.buf.ws) == 0
+        n_mean = float(np.mean(counts))
+        nbytes = 2.0 * h * d + 4.0 * n_mean * d  # per layer: W_gate + the kept W_up / W_down^T rows
+        us_l = t_sp * 1e3 / L
+        res[f"b{B}"] = {"us_per_step": round(t_sp * 1e3, 1), "us_per_layer": round(us_l, 2),
+                        "union_density": round(n_mean / h, 4),
+                        "achieved_gbs": round(nbytes / (us_l * 1e-6) / 1e9, 1),
+                        "dense_us_per_layer": round(t_de * 1e3 / L, 2),
+                        "speedup_vs_dense": round(t_de / t_sp, 3)}
+    del layers, ws16
+    torch.cuda.empty_cache()
+    return res
+
+
+def sirius_measure(torch, cs, stream, world, dev, rounds=3):
+    """Sirius round on LLaMA-3-70B-shaped layers (d 8192, h 28672, bf16, 1.41 GB each): 16 one-token
+    sparse drafts (csffn_cats_ffn_forward) then the dense verify of the 16-token chunk
+    (csffn_dense_ffn_forward), against 16 dense one-token steps.  Two layers are alternated so no
+    step reads weights an earlier one left in L2; times are per layer.  Thresholds from 512
+    calibration vectors.  effective_density: weight rows the round reads over those of the 16 dense
+    steps (stack.round_effective_density); draft_rel_l2 and top1_agreement compare each draft's output
+    with the verify's for the same token (top-1 of a fixed seeded projection to 64 values)."""
+    from contextual_sparsity_ffn_b200 import stack
+    d, h, T = 8192, 28672, 16
+    gen = torch.Generator(device=dev).manual_seed(4)
+    layers = [device_layer(torch, cs, d, h, gen, dev) for _ in range(2)]
+    xc = torch.randn(512, d, generator=gen, device=dev).to(torch.bfloat16)
+    x = torch.randn(T, d, generator=gen, device=dev).to(torch.bfloat16)
+    proj = torch.randn(d, 64, generator=gen, device=dev)
+    buf = cs.DecodeBuffers.new(layers[0], 1)
+    ws_dense = cs.new_workspace(layers[0], T)
+    sparse = torch.zeros(T, d, device=dev)
+    dense = torch.zeros(T, d, device=dev)
+    t_dev = torch.zeros(1, device=dev)
+
+    def dense_tokens(k):
+        for layer in layers:
+            for j in range(T):
+                cs.dense_ffn_forward(layer, x[j:j + 1], dense[j:j + 1], buf.ws)
+
+    g = run_graph_steps(torch, dense_tokens, rounds, 3, stream)
+    t_dense = max_over_ranks(time_graph_once(torch, g, stream), world, dev) / (rounds * len(layers))
+    del g
+    res = {"path": "16 x csffn_cats_ffn_forward (batch 1) + csffn_dense_ffn_forward (batch 16) per layer",
+           "dense_16_steps_us_per_layer": round(t_dense * 1e3, 1)}
+    for s in (0.5, 0.9):
+        ts = []
+        for layer in layers:
+            cs.calibrate_threshold(layer, xc, s, cs._abi.CAL_GLOBAL_ABS_ACT, t_dev)
+            ts.append(float(t_dev.item()))
+        rec = []
+        stack.sirius_round(layers[0], x, ts[0], sparse, dense, buf, ws_dense, record=rec)
+        counts = [len(idx) for idx, _ in rec]
+        rel = (torch.linalg.vector_norm(sparse - dense, dim=1) / torch.linalg.vector_norm(dense, dim=1))
+        top1 = (torch.argmax(sparse @ proj, dim=1) == torch.argmax(dense @ proj, dim=1)).float()
+
+        def round_step(k):
+            for layer, t in zip(layers, ts):
+                stack.sirius_round(layer, x, t, sparse, dense, buf, ws_dense)
+
+        g = run_graph_steps(torch, round_step, rounds, 3, stream)
+        t_round = max_over_ranks(time_graph_once(torch, g, stream), world, dev) / (rounds * len(layers))
+        del g
+        assert cs.check_status(buf.ws) == 0 and cs.check_status(ws_dense) == 0
+        res[f"s{int(round(s * 100))}"] = {
+            "us_per_round_per_layer": round(t_round * 1e3, 1),
+            "time_vs_16_dense_steps": round(t_round / t_dense, 4),
+            "neuron_density": round(float(np.mean(counts)) / h, 4),
+            "effective_density": round(stack.round_effective_density(counts, h), 4),
+            "draft_rel_l2_mean": round(float(rel.mean()), 4),
+            "top1_agreement": round(float(top1.mean()), 4)}
+    del layers, buf, ws_dense
+    torch.cuda.empty_cache()
+    return res
+
+
 def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
     """SVD-predictor ReGLU workload (d 4096, h 11008, bf16, per-neuron thresholds at q = 0.9):
     per step csffn_svd_ffn_forward (predictor, gate on the predicted set, up and down on the active
@@ -407,8 +541,9 @@ def csffn_arm(args, world, rank, local):
         return statistics.median(times)
 
     # ---- main measurement: K steps at the headline sparsity in one graph, events around the replay.
-    # No event nodes inside this graph: they add a gap before every launch.  With the one-launch path
-    # the average launch duration is the replay time / K (inter-launch gaps included).
+    # No event nodes inside this graph: they add a gap before every launch (and would break the
+    # programmatic dependency between a step's two kernels).  The average step duration is the
+    # replay time / K (gaps between steps included).
     g_main = run_graph_steps(torch, sparse_step(args.sparsity), K, W, stream)
     bus = pci_bus_id(torch, local)
     sampler = ClockSampler(bus).start()
@@ -459,8 +594,8 @@ def csffn_arm(args, world, rank, local):
         kern_name = "gate_stream_kernel (csffn_gate_mask)"
         kern_bytes = 2.0 * H * D + 2 * D + 8.0 * n_act
     else:
-        kern_name = "cats_ring_kernel (csffn_cats_ffn_forward)"
-        kern_bytes = step_bytes(n_act)  # the whole step is one kernel launch
+        kern_name = "cats_ring_kernel + ring_finish_kernel (csffn_cats_ffn_forward)"
+        kern_bytes = step_bytes(n_act)  # the step's two launches, taken together
     kern_gbs = kern_bytes / (kern_avg_us * 1e-6) / 1e9
 
     detail = {}
@@ -471,7 +606,7 @@ def csffn_arm(args, world, rank, local):
         u2 = whole_job_us_per_layer(t2, K, world)
         detail[f"{'two_call' if other else 'one_launch'}_{int(round(args.sparsity * 100))}"] = {
             "path": "csffn_gate_mask + csffn_sparse_ffn_forward (3 kernels)" if other
-                    else "csffn_cats_ffn_forward (1 kernel)", "us_per_layer": round(u2, 3),
+                    else "csffn_cats_ffn_forward (2 kernels)", "us_per_layer": round(u2, 3),
             "achieved_gbs": round(step_bytes(n_act) / (u2 * 1e-6) / 1e9, 1)}
         del g
         for s in sparsities[1:]:
@@ -505,6 +640,8 @@ def csffn_arm(args, world, rank, local):
         del g
         detail["dense_verify_70b_b16"] = dense_verify_measure(torch, cs, stream, K, W, world, dev)
         detail["svd_reglu_q90"] = svd_reglu_measure(torch, cs, synth, stream, K, world, dev)
+        detail["stack_llama3_8b_32_layers"] = stack_measure(torch, cs, stream, world, dev)
+        detail["sirius_round_70b"] = sirius_measure(torch, cs, stream, world, dev)
     del g_main
 
     # ---- end to end through the public API: pinned host x in, host out back, every step
@@ -535,10 +672,11 @@ def csffn_arm(args, world, rank, local):
                      "traffic": profiled_traffic(), "algorithmic_bytes_per_launch": round(kern_bytes),
                      "avg_launch_us": round(kern_avg_us, 3),
                      "timing": ("events around each csffn_gate_mask launch inside a graph" if HEADLINE_TWO_CALL else
-                                "events around each replay of the K-launch graph; per launch = median replay / K"),
+                                "events around each replay of the K-step graph; per step (its two launches and the gap "
+                                "between them) = median replay / K"),
                      "replays": spread.get("headline")},
         "e2e": e2e,
-        "gpu_launches": (3 if HEADLINE_TWO_CALL else 1) * K,
+        "gpu_launches": (3 if HEADLINE_TWO_CALL else 2) * K,
         "clocks": clocks,
     }
     if detail:

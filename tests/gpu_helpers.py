@@ -4,6 +4,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+import oracle
 from contextual_sparsity_ffn_b200 import binding as cs
 
 DEV = "cuda"
@@ -73,3 +74,12 @@ def assert_index_list(idx: np.ndarray, h: int) -> None:
     assert idx.dtype == np.int32
     assert np.all(idx >= 0) and np.all(idx < h)
     assert np.all(np.diff(idx) > 0), "indices must be unique and ascending"
+
+
+def check_values(a_val, idx, a_ref, m, t):
+    """a_val against the oracle's activations, element by element: a where the token keeps the row,
+    0 where it rejects it; the per-token masks agree with the oracle's outside the band."""
+    tb = np.abs(np.abs(a_ref) - t) < 1e-3 * abs(t)
+    assert np.array_equal(m[~tb], oracle.cats_mask(a_ref, t)[~tb])
+    np.testing.assert_allclose(a_val, np.where(m, a_ref, 0.0)[:, idx], rtol=1e-4,
+                               atol=1e-6 * np.abs(a_ref).max())

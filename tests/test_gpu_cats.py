@@ -13,8 +13,8 @@ import oracle
 from contextual_sparsity_ffn_b200 import synth
 from contextual_sparsity_ffn_b200 import binding as cs
 
-from gpu_helpers import (assert_index_list, band_rows, dev, dev_layer, run_dense, run_gate, run_sparse,
-                         token_masks)
+from gpu_helpers import (assert_index_list, band_rows, check_values, dev, dev_layer, run_dense, run_gate,
+                         run_sparse, token_masks)
 
 pytestmark = pytest.mark.gpu
 
@@ -239,15 +239,6 @@ def test_dense_token_block_tensor_cores(d, h, B, act):
 
 
 # ------------------------------------------------------------------------------ one-launch decode step
-
-def check_values(a_val, idx, a_ref, m, t):
-    """a_val against the oracle's activations, element by element: a where the token keeps the row,
-    0 where it rejects it; the per-token masks agree with the oracle's outside the band."""
-    tb = np.abs(np.abs(a_ref) - t) < 1e-3 * abs(t)
-    assert np.array_equal(m[~tb], oracle.cats_mask(a_ref, t)[~tb])
-    np.testing.assert_allclose(a_val, np.where(m, a_ref, 0.0)[:, idx], rtol=1e-4,
-                               atol=1e-6 * np.abs(a_ref).max())
-
 
 def run_fused(layer, x_np, t, out_dtype=torch.float32, ws=None):
     x = dev(x_np if x_np.ndim == 2 else x_np[None, :])
