@@ -205,6 +205,27 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
 
 namespace {
 
+// Arguments of the tensor-core FFN (tc_ffn.cu) for this layer, tokens and workspace.
+TcArgs tc_args(const csffn_layer* layer, const void* x, int B, const WsLayout& L, void* ws) {
+  TcArgs a{};
+  a.W_gate = layer->w_gate;
+  a.W_up = layer->w_up;
+  a.W_down_t = layer->w_down_t;
+  a.x = x;
+  a.d = layer->d;
+  a.h = layer->h;
+  a.B = B;
+  a.bias = layer->gate_bias;
+  a.act = layer->act;
+  a.v = at<uint16_t>(ws, L.vbuf);
+  a.afull = at<float>(ws, L.afull);
+  a.flags = at<uint8_t>(ws, L.flags);
+  a.part = at<float>(ws, L.tcpart);
+  a.ctr = at<uint32_t>(ws, L.tcctr);
+  a.err = at<uint32_t>(ws, L.err);
+  return a;
+}
+
 // Every check of a CATS step with 1 <= B <= CSFFN_MAX_BATCH, whichever path runs it (the one-launch
 // kernel, or the gate mask then the gathered up/down), so that a rejected call launches nothing.
 csffn_status check_cats_step(const csffn_layer* layer, const void* x, int B, float t, const int32_t* idx,
@@ -214,6 +235,7 @@ csffn_status check_cats_step(const csffn_layer* layer, const void* x, int B, flo
   if (st != CSFFN_OK) return st;
   if (!aligned16(x) || !aligned16(out)) return CSFFN_ERR_ALIGNMENT;
   if (!cats_ring_supported(layer->d, B, layer->wdtype) && !cats_fused_supported(layer->d, B, layer->wdtype) &&
+      !tc_ffn_supported(layer->d, layer->h, B, layer->wdtype) &&
       (size_t)batch_tier(B) * layer->d * esize(layer->wdtype) > kMaxDynSmem)
     return CSFFN_ERR_UNSUPPORTED_SHAPE;
   return check_ws(ws, ws_bytes, ws_layout(layer->d, layer->h, B, 0).ybuf);
@@ -235,6 +257,20 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
   if ((st = check_cats_step(layer, x, B, t, idx, a_val, out, ws, ws_bytes)) != CSFFN_OK) return st;
   const bool ring = cats_ring_supported(layer->d, B, layer->wdtype);
+  if (!ring && !cand_idx && tc_ffn_supported(layer->d, layer->h, B, layer->wdtype)) {
+    // Batches past the streaming step's tiers: the union of the tokens' masks covers most neurons,
+    // so every row is read once by the tensor cores with the rejected activations zeroed.
+    const WsLayout L = ws_layout(layer->d, layer->h, B, 0);
+    TcArgs a = tc_args(layer, x, B, L, ws);
+    a.masked = 1;
+    a.t = t;
+    a.idx = idx;
+    a.count = count;
+    a.a_val = a_val;
+    a.out = out;
+    a.out_mode = out_mode;
+    return cuda_status(launch_tc_ffn(a, as_stream(stream)));
+  }
   if (!ring && !cats_fused_supported(layer->d, B, layer->wdtype)) {
     st = csffn_gate_mask(layer, x, B, t, cand_idx, cand_count, idx, count, a_val, ws, ws_bytes, stream);
     if (st != CSFFN_OK) return st;
@@ -358,6 +394,12 @@ csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, in
   if ((st = check_ws(ws, ws_bytes, L.ybuf)) != CSFFN_OK) return st;
   cudaStream_t s = as_stream(stream);
 
+  if (tc_ffn_supported(layer->d, layer->h, B, layer->wdtype)) {  // fifth-generation tensor cores
+    TcArgs a = tc_args(layer, x, B, L, ws);
+    a.out = out;
+    a.out_mode = out_mode;
+    return cuda_status(launch_tc_ffn(a, s));
+  }
   if (dense_mma_supported(layer->d, layer->h, B, layer->wdtype)) {  // tensor cores, one pass
     DenseGateUpArgs g{};
     g.W_gate = layer->w_gate;

@@ -42,11 +42,13 @@ struct WsLayout {
   size_t tickets;    // uint32 [64][32]                 chunk-ticket counters, 128 B apart (fused path)
   size_t facc;       // fp32 [kFusedAccCopies][kFusedMaxBatch][CSFFN_MAX_D] out accumulators (fused path)
   size_t status;     // uint64 [kNumCtl][max_chunks]   look-back status words
+  size_t tcctr;      // uint32 [tc_counters(h)]         k-blocks done per tile (tensor-core FFN)
   size_t control_end;
   size_t vbuf;       // fp32 [max_batch][h]            v = a * u (sparse) or act(z)*u (dense)
   size_t afull;      // fp32 [max_batch][h]            per-neuron kept activations (fused path)
   size_t flags;      // uint8 [h]                      per-neuron keep flags (fused path)
   size_t partial;    // fp32 [partial_rows(max_batch)][d]
+  size_t tcpart;     // fp32 [kTcMaxCtas][2][32][128]    split tiles' partial accumulators (tensor-core FFN)
   size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
   size_t hx;         // [max_batch][d] (4 B each)      tokens staged from host memory (host entry point)
   size_t hout;       // fp32 [max_batch][d]            output staged for the copy back to host memory
@@ -57,6 +59,12 @@ struct WsLayout {
 constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
 constexpr int kFusedMaxBatch = 4;
 constexpr int kFusedAccCopies = 4;  // fused step: CTA k adds into accumulator k % kFusedAccCopies
+
+// Tensor-core FFN (tc_ffn.cu): tiles of 128 neurons (gate/up) or 128 output columns (down); at most
+// kTcMaxCtas CTAs, each with two partial-accumulator slots of 32 x 128 floats.
+constexpr int kTcTile = 128;
+constexpr int kTcMaxCtas = 160;
+__host__ __device__ inline int tc_counters(int h) { return (h + kTcTile - 1) / kTcTile + CSFFN_MAX_D / kTcTile; }
 
 // Rows of d floats in the partial region (one per row range of the sparse/dense forward).
 __host__ __device__ inline int partial_rows(int max_batch) { return kMaxRowRanges * max_batch; }
@@ -77,6 +85,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   L.max_chunks = (h + kChunkRows - 1) / kChunkRows;
   L.status = o;     o += sizeof(uint64_t) * (size_t)kNumCtl * L.max_chunks;
   o = align_up(o, 256);
+  L.tcctr = o;      o += sizeof(uint32_t) * (size_t)tc_counters(h);
+  o = align_up(o, 256);
   L.control_end = o;
   L.vbuf = o;       o += sizeof(float) * (size_t)max_batch * h;
   o = align_up(o, 256);
@@ -86,6 +96,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   o = align_up(o, 256);
   // partials: one per row range of the sparse/dense forward
   L.partial = o;    o += sizeof(float) * (size_t)partial_rows(max_batch) * d;
+  o = align_up(o, 256);
+  L.tcpart = o;     o += sizeof(float) * (size_t)kTcMaxCtas * 2 * 32 * kTcTile;
   o = align_up(o, 256);
   L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);
   o = align_up(o, 256);

@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 #include "tma.cuh"
 
 namespace csffn {
@@ -341,10 +342,7 @@ cudaError_t launch_dense_gate_up_mma(const DenseGateUpArgs& a, cudaStream_t s) {
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link against libcuda).
-typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-static TensorMapEncodeFn tensor_map_encoder() {
+TensorMapEncodeFn tensor_map_encoder() {
   static TensorMapEncodeFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;

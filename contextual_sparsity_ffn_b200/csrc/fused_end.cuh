@@ -71,18 +71,83 @@ __device__ __forceinline__ int step_neuron(const int32_t* cand, int h, int j) {
   return (unsigned)r < (unsigned)h ? r : 0;
 }
 
+// Compaction of a step's keep flags into idx / a_val / count, by 128 threads of every CTA of the
+// grid (ct = 0 .. 127 their index, named barrier `bar` among them): CTA k owns a fixed range of
+// 32-position words, counts the kept positions before it from the flag bytes (each 0 or 1, so a
+// 32-bit word's popcount counts its kept rows) and writes its positions' neurons and kept
+// activations in ascending order; the last CTA writes the count.
+template <int NB>
+__device__ __forceinline__ void compact_flags(const FusedArgs& p, int n_rows, uint32_t* s_cnt, int ct, int bar) {
+  const int lane = ct & 31, cw = ct >> 5;
+  const int B = p.B, h = p.h;
+  const int n_words = (n_rows + kWarp - 1) / kWarp;
+  const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
+  const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
+  if (!(wa < wb || blockIdx.x == gridDim.x - 1)) return;
+  bool f;
+  int nr;
+  float av[NB];
+  auto load_pass = [&](int w0) {  // flag, neuron and activations of position (w0 + cw) * 32 + lane
+    const int jp = (w0 + cw) * kWarp + lane;
+    const bool in = w0 + cw < wb && jp < n_rows;
+    f = in && __ldcg(p.flags + jp) != 0;
+    nr = in ? step_neuron(p.cand_idx, h, jp) : 0;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
+  };
+  load_pass(wa);
+  uint32_t before = 0;
+  const uint4* f4 = reinterpret_cast<const uint4*>(p.flags);
+  for (int i0 = ct; i0 < wa * 2; i0 += kFinishHalf * kCountLoads) {  // each batch's loads issued together
+    uint4 fw[kCountLoads];
+#pragma unroll
+    for (int u = 0; u < kCountLoads; ++u)
+      fw[u] = i0 + u * kFinishHalf < wa * 2 ? __ldcg(f4 + i0 + u * kFinishHalf) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kCountLoads; ++u)
+      before += __popc(fw[u].x) + __popc(fw[u].y) + __popc(fw[u].z) + __popc(fw[u].w);
+  }
+  before = warp_sum_u32(before);
+  if (lane == 0) s_cnt[cw] = before;
+  named_sync(bar, kFinishHalf);
+  uint32_t base = 0;
+#pragma unroll
+  for (int w = 0; w < kFinishHalf / kWarp; ++w) base += s_cnt[w];
+  named_sync(bar, kFinishHalf);
+  for (int w0 = wa; w0 < wb; w0 += kFinishHalf / kWarp) {
+    const uint32_t m = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) s_cnt[cw] = __popc(m);
+    named_sync(bar, kFinishHalf);
+    uint32_t off = base, total = base;
+#pragma unroll
+    for (int ww = 0; ww < kFinishHalf / kWarp; ++ww) {
+      off += ww < cw ? s_cnt[ww] : 0u;
+      total += s_cnt[ww];
+    }
+    if (f) {
+      const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
+      p.idx[pos] = nr;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (b < B) p.a_val[(size_t)b * h + pos] = av[b];
+    }
+    base = total;
+    named_sync(bar, kFinishHalf);
+    load_pass(w0 + kFinishHalf / kWarp);
+  }
+  if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
+}
+
 // The end phase, called by every thread of the CTA (blockDim.x >= 2 * kFinishHalf) once every CTA's
 // partial output is in the accumulators and every keep flag is written (after the meeting below, or
 // in a kernel that follows the one that wrote them).  Threads [0, kFinishHalf) write out (the sum of
 // the accumulators, plus the old out when accumulating) over an equal share of the columns and
 // clear the accumulators for the next launch; threads [kFinishHalf, 2 kFinishHalf) compact idx /
-// a_val / count from the keep flags: CTA k owns a fixed range of 32-position words, counts the kept
-// positions before it from the flag bytes (each 0 or 1, so a 32-bit word's popcount counts its
-// kept rows) and writes its positions' neurons in ascending order.
+// a_val / count from the keep flags (compact_flags, named barrier 2).
 template <int NB>
 __device__ void fused_finish_work(const FusedArgs& p, int n_rows, uint32_t* s_cnt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int B = p.B, d = p.d, h = p.h;
+  const int tid = threadIdx.x;
+  const int B = p.B, d = p.d;
   if (tid < kFinishHalf) {
     const int n4 = B * d / 4;
     const int i0 = (int)((long long)n4 * blockIdx.x / gridDim.x);
@@ -122,64 +187,7 @@ __device__ void fused_finish_work(const FusedArgs& p, int n_rows, uint32_t* s_cn
         __stcg(reinterpret_cast<float4*>(p.facc + (size_t)c * B * d) + i, make_float4(0.f, 0.f, 0.f, 0.f));
     }
   } else if (tid < 2 * kFinishHalf) {
-    const int ct = tid - kFinishHalf, cw = warp - kFinishHalf / kWarp;
-    const int n_words = (n_rows + kWarp - 1) / kWarp;
-    const int wa = (int)((long long)n_words * blockIdx.x / gridDim.x);
-    const int wb = (int)((long long)n_words * (blockIdx.x + 1) / gridDim.x);
-    if (wa < wb || blockIdx.x == gridDim.x - 1) {
-      bool f;
-      int nr;
-      float av[NB];
-      auto load_pass = [&](int w0) {  // flag, neuron and activations of position (w0 + cw) * 32 + lane
-        const int jp = (w0 + cw) * kWarp + lane;
-        const bool in = w0 + cw < wb && jp < n_rows;
-        f = in && __ldcg(p.flags + jp) != 0;
-        nr = in ? step_neuron(p.cand_idx, h, jp) : 0;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) av[b] = (in && b < B) ? __ldcg(p.afull + (size_t)b * h + jp) : 0.f;
-      };
-      load_pass(wa);
-      uint32_t before = 0;
-      const uint4* f4 = reinterpret_cast<const uint4*>(p.flags);
-      for (int i0 = ct; i0 < wa * 2; i0 += kFinishHalf * kCountLoads) {  // each batch's loads issued together
-        uint4 fw[kCountLoads];
-#pragma unroll
-        for (int u = 0; u < kCountLoads; ++u)
-          fw[u] = i0 + u * kFinishHalf < wa * 2 ? __ldcg(f4 + i0 + u * kFinishHalf) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int u = 0; u < kCountLoads; ++u)
-          before += __popc(fw[u].x) + __popc(fw[u].y) + __popc(fw[u].z) + __popc(fw[u].w);
-      }
-      before = warp_sum_u32(before);
-      if (lane == 0) s_cnt[cw] = before;
-      named_sync(2, kFinishHalf);
-      uint32_t base = 0;
-#pragma unroll
-      for (int w = 0; w < kFinishHalf / kWarp; ++w) base += s_cnt[w];
-      named_sync(2, kFinishHalf);
-      for (int w0 = wa; w0 < wb; w0 += kFinishHalf / kWarp) {
-        const uint32_t m = __ballot_sync(0xffffffffu, f);
-        if (lane == 0) s_cnt[cw] = __popc(m);
-        named_sync(2, kFinishHalf);
-        uint32_t off = base, total = base;
-#pragma unroll
-        for (int ww = 0; ww < kFinishHalf / kWarp; ++ww) {
-          off += ww < cw ? s_cnt[ww] : 0u;
-          total += s_cnt[ww];
-        }
-        if (f) {
-          const uint32_t pos = off + __popc(m & ((1u << lane) - 1u));
-          p.idx[pos] = nr;
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-            if (b < B) p.a_val[(size_t)b * h + pos] = av[b];
-        }
-        base = total;
-        named_sync(2, kFinishHalf);
-        load_pass(w0 + kFinishHalf / kWarp);
-      }
-      if (blockIdx.x == gridDim.x - 1 && ct == 0) *p.count = (int32_t)base;
-    }
+    compact_flags<NB>(p, n_rows, s_cnt, tid - kFinishHalf, 2);
   }
 }
 

@@ -144,6 +144,38 @@ cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
 bool cats_ring_supported(int d, int B, int wdtype);
 cudaError_t launch_cats_ring(const FusedArgs& a, int wdtype, cudaStream_t s);
 
+// Gated FFN of up to 16 tokens on the fifth-generation tensor cores (tc_ffn.cu): a gate/up kernel
+// (tcgen05.mma, operands staged by TMA tensor copies, fp32 accumulators in TMEM) writes v = act(z +
+// beta) * u as bf16 high and low parts, then a down kernel (the same machinery, W_down^T read
+// MN-major) writes out.  Both split their work evenly over the SMs as contiguous runs of 64-element
+// k-blocks (a tile split between CTAs is finished by the last one to arrive).  Masked mode is the
+// CATS step: v and the kept activations are zero where |act(z + beta)| <= t, the keep flags are
+// written, and the down kernel also compacts idx / a_val / count.
+struct TcArgs {
+  const void* W_gate;
+  const void* W_up;
+  const void* W_down_t;
+  const void* x;      // [B, d] bf16
+  int d, h, B;
+  const float* bias;  // [h] or NULL
+  int act;
+  int masked;         // CATS step (flags, afull, idx / a_val / count written)
+  float t;
+  uint16_t* v;        // [2][B][h] bf16 bits: high parts, then low parts
+  float* afull;       // [B, h] kept activations (masked)
+  uint8_t* flags;     // [h] keep flags (masked)
+  float* part;        // [kTcMaxCtas][2][32][128] partial accumulators
+  uint32_t* ctr;      // [tc_counters(h)]: gate/up tiles, then down column tiles; zero between launches
+  uint32_t* err;
+  int32_t* idx;       // masked: the compacted union (as csffn_cats_ffn_forward)
+  int32_t* count;
+  float* a_val;
+  void* out;
+  int out_mode;
+};
+bool tc_ffn_supported(int d, int h, int B, int wdtype);
+cudaError_t launch_tc_ffn(const TcArgs& a, cudaStream_t s);
+
 // Radix selection and per-neuron selection (calibration).
 size_t kth_state_bytes();
 cudaError_t launch_kth_smallest(const float* values, int64_t n, int64_t k, float* out, void* state,

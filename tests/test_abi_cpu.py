@@ -177,9 +177,10 @@ def test_one_launch_step_validation(lib):
     assert call(L=bad_down) == _abi.ERR_ALIGNMENT
     assert call(ws=0) == _abi.ERR_WORKSPACE
     assert call(ws_bytes=1 << 20) == _abi.ERR_WORKSPACE
-    # shapes the one-launch kernel does not take go to the two-call path, whose own limits hold too
-    assert call(L=layer(d=16384), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
-    assert call(L=layer(d=16384), B=16, idx=0) == _abi.ERR_INVALID_ARG
+    # shapes neither the one-launch kernels nor the tensor-core path take (d not a multiple of 64) go
+    # to the two-call path, whose own limits hold too
+    assert call(L=layer(d=16376), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
+    assert call(L=layer(d=16376), B=16, idx=0) == _abi.ERR_INVALID_ARG
     assert call(L=layer(d=4100)) == _abi.ERR_ALIGNMENT
 
 
@@ -203,7 +204,7 @@ def test_host_buffer_step_validation(lib):
     no_gate.w_gate = None
     assert call(L=no_gate) == _abi.ERR_INVALID_ARG
     assert call(ws_bytes=1 << 20) == _abi.ERR_WORKSPACE  # the staging buffers are part of the workspace
-    assert call(L=layer(d=16384), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
+    assert call(L=layer(d=16376), B=16) == _abi.ERR_UNSUPPORTED_SHAPE
 
 
 def test_predictor_step_validation(lib):
