@@ -399,9 +399,11 @@ def sirius_measure(torch, cs, stream, world, dev, rounds=3):
 
 def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
     """SVD-predictor ReGLU workload (d 4096, h 11008, bf16, per-neuron thresholds at q = 0.9):
-    per step csffn_svd_ffn_forward (predictor, gate on the predicted set, up and down on the active
-    set: one launch); us_two_calls times csffn_predict_lowrank + csffn_cats_ffn_forward on the
-    predicted set for the same tokens.  This step reads a few tens of MB, less than L2,
+    per step csffn_svd_ffn_forward (y = x U_r, one grid-wide count, then predictor, gate on the
+    predicted set, up and down on the active set: one cooperative launch); "parallel" times
+    csffn_svd_ffn_forward_parallel (W_up read with
+    W_gate on the predicted set); us_two_calls times csffn_predict_lowrank + csffn_cats_ffn_forward
+    on the predicted set for the same tokens.  This step reads a few tens of MB, less than L2,
     so L2 is flushed (a 256 MB write) before every step: step time = time of K x (flush + step)
     minus time of K x flush, both as one CUDA graph.  The truncated SVD of W_gate is the offline
     stage (outside the library), done here with torch on the device."""
@@ -435,6 +437,10 @@ def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
             x1 = xs[k % N_TOKENS: k % N_TOKENS + 1]
             cs.svd_ffn_forward(layer, x1, urt, vr, tau, 0.0, idx, cnt, av, o, ws)
 
+        def step_par(k):
+            x1 = xs[k % N_TOKENS: k % N_TOKENS + 1]
+            cs.svd_ffn_forward(layer, x1, urt, vr, tau, 0.0, idx, cnt, av, o, ws, parallel=True)
+
         n_p, n_a = [], []
         for k in range(min(n, N_TOKENS)):
             step_two(k)
@@ -460,18 +466,25 @@ def svd_reglu_measure(torch, cs, synth, stream, K, world, dev):
 
         t_flush = timed(None)
         us = max_over_ranks(timed(step) - t_flush, world, dev)
+        us_par = max_over_ranks(timed(step_par) - t_flush, world, dev)
         us_two = max_over_ranks(timed(step_two) - t_flush, world, dev)
         mp, ma = float(np.mean(n_p)), float(np.mean(n_a))
+        # U_r, V_r, the predicted rows' W_gate, the kept rows' W_up and W_down^T (parallel: W_up of
+        # every predicted row), flags and index lists
         nbytes = (r * D + H * r) * 2 + mp * D * 2 + 2 * ma * D * 2 + mp * 4 + ma * 8
+        nbytes_par = (r * D + H * r) * 2 + 2 * mp * D * 2 + ma * D * 2 + mp * 4 + ma * 8
         out_d[f"r{r}"] = {"us_per_layer": round(us, 2), "predicted_rows": round(mp, 1), "active_rows": round(ma, 1),
                           "bytes_needed_mb": round(nbytes / 1e6, 2),
                           "achieved_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
                           "launches_per_step": 1,
+                          "parallel": {"us_per_layer": round(us_par, 2), "bytes_needed_mb": round(nbytes_par / 1e6, 2),
+                                       "achieved_gbs": round(nbytes_par / (us_par * 1e-6) / 1e9, 1)},
                           "us_two_calls": round(us_two, 2)}
         del ws
     del flush, layer
     torch.cuda.empty_cache()
-    out_d["path"] = "csffn_svd_ffn_forward (one launch); L2 flushed before every step"
+    out_d["path"] = ("csffn_svd_ffn_forward (one cooperative launch); csffn_svd_ffn_forward_parallel beside it; "
+                     "L2 flushed before every step")
     return out_d
 
 

@@ -54,6 +54,7 @@ SIGNATURES = {
     "csffn_cats_ffn_forward": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "csffn_cats_ffn_forward_host": (_I, [_L, _P, _I, _F, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "csffn_svd_ffn_forward": (_I, [_L, _P, _I, _I, _P, _P, _P, _F, _P, _P, _P, _P, _I, _P, _Z, _P]),
+    "csffn_svd_ffn_forward_parallel": (_I, [_L, _P, _I, _I, _P, _P, _P, _F, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "csffn_predict_lowrank": (_I, [_L, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "csffn_calibrate_workspace_size": (_Z, [_L, _I, _I, _I]),
     "csffn_calibrate_threshold": (_I, [_L, _P, _I, _F, _I, _P, _P, _I, _P, _P, _Z, _P]),

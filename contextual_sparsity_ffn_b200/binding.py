@@ -205,15 +205,17 @@ def predict_lowrank(layer: FFNLayer, x: torch.Tensor, u_rt: torch.Tensor, v_r: t
 
 def svd_ffn_forward(layer: FFNLayer, x: torch.Tensor, u_rt: torch.Tensor, v_r: torch.Tensor, tau: torch.Tensor,
                     t: float, idx: torch.Tensor, count: torch.Tensor, a_val: torch.Tensor, out: torch.Tensor,
-                    ws: torch.Tensor, out_mode: Optional[int] = None, stream=None) -> None:
+                    ws: torch.Tensor, out_mode: Optional[int] = None, stream=None, parallel: bool = False) -> None:
+    """csffn_svd_ffn_forward, or with parallel=True csffn_svd_ffn_forward_parallel (same outputs)."""
     B = x.shape[0] if x.dim() == 2 else 1
     rank = u_rt.shape[0]
     if out_mode is None:
         out_mode = _abi.OUT_BF16 if out.dtype == torch.bfloat16 else _abi.OUT_F32
-    check(load().csffn_svd_ffn_forward(layer.ref(), _ptr(x), B, rank, _ptr(u_rt), _ptr(v_r), _ptr(tau), float(t),
-                                       _ptr(idx), _ptr(count), _ptr(a_val), _ptr(out), out_mode, _ptr(ws),
-                                       _nbytes(ws), _stream(stream)),
-          "csffn_svd_ffn_forward")
+    name = "csffn_svd_ffn_forward_parallel" if parallel else "csffn_svd_ffn_forward"
+    check(getattr(load(), name)(layer.ref(), _ptr(x), B, rank, _ptr(u_rt), _ptr(v_r), _ptr(tau), float(t),
+                                _ptr(idx), _ptr(count), _ptr(a_val), _ptr(out), out_mode, _ptr(ws), _nbytes(ws),
+                                _stream(stream)),
+          name)
 
 
 def calibrate_workspace_size(layer: FFNLayer, n: int, mode: int, rank: int = 0) -> int:

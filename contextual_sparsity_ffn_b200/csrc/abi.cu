@@ -256,10 +256,12 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
   if ((cand_idx == nullptr) != (cand_count == nullptr)) return CSFFN_ERR_INVALID_ARG;
   if (B == 0) return cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), as_stream(stream)));
   if ((st = check_cats_step(layer, x, B, t, idx, a_val, out, ws, ws_bytes)) != CSFFN_OK) return st;
-  const bool ring = cats_ring_supported(layer->d, B, layer->wdtype);
-  if (!ring && !cand_idx && tc_ffn_supported(layer->d, layer->h, B, layer->wdtype)) {
-    // Batches past the streaming step's tiers: the union of the tokens' masks covers most neurons,
-    // so every row is read once by the tensor cores with the rejected activations zeroed.
+  // From three tokens on, the union of the tokens' masks covers most neurons (about 1 - s^B of them
+  // at sparsity s), so every row is read once by the tensor cores with the rejected activations
+  // zeroed; that takes no longer than the streaming step even at 90% sparsity.
+  const bool tc = !cand_idx && tc_ffn_supported(layer->d, layer->h, B, layer->wdtype);
+  const bool ring = cats_ring_supported(layer->d, B, layer->wdtype) && !(tc && batch_tier(B) >= 4);
+  if (!ring && tc) {
     const WsLayout L = ws_layout(layer->d, layer->h, B, 0);
     TcArgs a = tc_args(layer, x, B, L, ws);
     a.masked = 1;
@@ -305,9 +307,11 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
                           : launch_cats_fused(a, layer->wdtype, as_stream(stream)));
 }
 
-csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
-                                   const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
-                                   float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+csffn_status svd_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt, const void* v_r,
+                         const float* tau, float t, bool parallel, int32_t* idx, int32_t* count, float* a_val,
+                         void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
   csffn_status st = check_layer_shape(layer);
   if (st != CSFFN_OK) return st;
   if (B < 0 || B > CSFFN_MAX_BATCH) return CSFFN_ERR_INVALID_ARG;
@@ -320,7 +324,9 @@ csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int 
   if (rank % vec_elems(layer->wdtype) != 0) return CSFFN_ERR_ALIGNMENT;
   if ((st = check_weights(layer, true, true, true)) != CSFFN_OK) return st;
   if (!aligned16(x) || !aligned16(out) || !aligned16(u_rt) || !aligned16(v_r)) return CSFFN_ERR_ALIGNMENT;
-  if (!cats_fused_supported(layer->d, B, layer->wdtype, rank)) return CSFFN_ERR_UNSUPPORTED_SHAPE;
+  const bool two = svd_step_supported(layer->d, layer->h, B, layer->wdtype, rank);
+  if (!two && (parallel || !cats_fused_supported(layer->d, B, layer->wdtype, rank)))
+    return CSFFN_ERR_UNSUPPORTED_SHAPE;
   const WsLayout L = ws_layout(layer->d, layer->h, B, rank);
   if ((st = check_ws(ws, ws_bytes, L.hx)) != CSFFN_OK) return st;
   FusedArgs a{};
@@ -344,13 +350,32 @@ csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int 
   a.facc = at<float>(ws, L.facc);
   a.ctl = reinterpret_cast<uint32_t*>(at<Control>(ws, L.ctl) + kCtlFused);
   a.tickets = at<uint32_t>(ws, L.tickets);
+  a.svd_counts = at<uint32_t>(ws, L.svdcnt);
   a.err = at<uint32_t>(ws, L.err);
   a.idx = idx;
   a.count = count;
   a.a_val = a_val;
   a.out = out;
   a.out_mode = out_mode;
+  if (two) return cuda_status(launch_svd_step(a, layer->wdtype, parallel, as_stream(stream)));
   return cuda_status(launch_cats_fused(a, layer->wdtype, as_stream(stream)));
+}
+
+}  // namespace
+
+csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
+                                   const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
+                                   float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream) {
+  return svd_forward(layer, x, B, rank, u_rt, v_r, tau, t, false, idx, count, a_val, out, out_mode, ws, ws_bytes,
+                     stream);
+}
+
+csffn_status csffn_svd_ffn_forward_parallel(const csffn_layer* layer, const void* x, int B, int rank,
+                                            const void* u_rt, const void* v_r, const float* tau, float t,
+                                            int32_t* idx, int32_t* count, float* a_val, void* out, int out_mode,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  return svd_forward(layer, x, B, rank, u_rt, v_r, tau, t, true, idx, count, a_val, out, out_mode, ws, ws_bytes,
+                     stream);
 }
 
 csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,

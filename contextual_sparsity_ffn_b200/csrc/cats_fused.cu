@@ -143,48 +143,9 @@ struct Tickets {
   }
 };
 
-// acc[b] += W[row] . x_b over this lane's share, row and tokens both in shared memory.
-template <typename WT, int NB>
-__device__ __forceinline__ void smem_row_dot(const WT* row, const WT* xs, int K, int lane, float (&acc)[NB]) {
-  constexpr int EPV = Vec<WT>::N;
-  const int NV = K / EPV;
-#pragma unroll 4
-  for (int v = lane; v < NV; v += kWarp) {
-    const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)v * EPV);
-    float wf[EPV];
-    unpack(w, wf);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      float xf[EPV];
-      load_x<EPV>(xs + (size_t)b * K + (size_t)v * EPV, xf);
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) acc[b] = fmaf(wf[e], xf[e], acc[b]);
-    }
-  }
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// acc[b] += row[0 .. n) . y_b[0 .. n): a row in shared memory against fp32 vectors y_b = ys + b * n.
-template <typename WT, int NB>
-__device__ __forceinline__ void smem_dot_f32(const WT* row, const float* ys, int n, int lane, float (&acc)[NB]) {
-  constexpr int EPV = Vec<WT>::N;
-  const int nv = n / EPV;
-#pragma unroll 4
-  for (int v = lane; v < nv; v += kWarp) {
-    float wf[EPV];
-    unpack(*reinterpret_cast<const uint4*>(row + (size_t)v * EPV), wf);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      float yf[EPV];
-      load_x<EPV>(ys + (size_t)b * n + (size_t)v * EPV, yf);
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) acc[b] = fmaf(wf[e], yf[e], acc[b]);
-    }
-  }
-}
-
 // PRED: predictor mode ("SVD Contextual Sparsity Predictors for Fast LLM Inference", Fig. 1 and
 // Fig. 3).  Before the chunk loop the grid computes y = x U_r (a warp per row of U_r^T) and meets
 // at a grid-wide count; the chunks then prefetch rows of V_r instead of W_gate, each warp forms

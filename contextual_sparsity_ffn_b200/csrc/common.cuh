@@ -49,6 +49,7 @@ struct WsLayout {
   size_t flags;      // uint8 [h]                      per-neuron keep flags (fused path)
   size_t partial;    // fp32 [partial_rows(max_batch)][d]
   size_t tcpart;     // fp32 [kTcMaxCtas][2][32][128]    split tiles' partial accumulators (tensor-core FFN)
+  size_t svdcnt;     // uint32 [kTcMaxCtas]              kept rows per CTA (SVD step)
   size_t ybuf;       // fp32 [max_batch][max_rank]     predictor y = x U_r
   size_t hx;         // [max_batch][d] (4 B each)      tokens staged from host memory (host entry point)
   size_t hout;       // fp32 [max_batch][d]            output staged for the copy back to host memory
@@ -98,6 +99,8 @@ inline WsLayout ws_layout(int d, int h, int max_batch, int max_rank) {
   L.partial = o;    o += sizeof(float) * (size_t)partial_rows(max_batch) * d;
   o = align_up(o, 256);
   L.tcpart = o;     o += sizeof(float) * (size_t)kTcMaxCtas * 2 * 32 * kTcTile;
+  o = align_up(o, 256);
+  L.svdcnt = o;     o += sizeof(uint32_t) * (size_t)kTcMaxCtas;
   o = align_up(o, 256);
   L.ybuf = o;       o += sizeof(float) * (size_t)max_batch * (max_rank > 0 ? max_rank : 1);
   o = align_up(o, 256);

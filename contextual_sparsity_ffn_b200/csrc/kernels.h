@@ -130,6 +130,7 @@ struct FusedArgs {
   float* facc;      // fp32 [kFusedAccCopies][B, d] accumulators of out, zero between launches
   uint32_t* ctl;     // fused control words (arrival counter, generation), zero before first use
   uint32_t* tickets; // [32 * 32] chunk-ticket counters and dry flags, 128 bytes apart
+  uint32_t* svd_counts;  // [kTcMaxCtas] SVD step: kept rows per CTA
   uint32_t* err;
   int32_t* idx;
   int32_t* count;
@@ -143,6 +144,12 @@ cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
 // bulk copies from one producer warp (ring.cu): one CTA per SM.
 bool cats_ring_supported(int d, int B, int wdtype);
 cudaError_t launch_cats_ring(const FusedArgs& a, int wdtype, cudaStream_t s);
+
+// SVD-predicted step of up to 4 tokens in one cooperative launch (svd_step.cu): y = x U_r, one
+// grid-wide count, then predictor, gate, up, down and the end phase; `parallel` fetches W_up with
+// W_gate for the predicted rows.
+bool svd_step_supported(int d, int h, int B, int wdtype, int rank);
+cudaError_t launch_svd_step(const FusedArgs& a, int wdtype, bool parallel, cudaStream_t s);
 
 // Gated FFN of up to 16 tokens on the fifth-generation tensor cores (tc_ffn.cu): a gate/up kernel
 // (tcgen05.mma, operands staged by TMA tensor copies, fp32 accumulators in TMEM) writes v = act(z +

@@ -144,23 +144,28 @@ csffn_status csffn_sparse_ffn_forward(const csffn_layer* layer, const void* x, i
                                       const int32_t* idx, const int32_t* count, const float* a_val,
                                       void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
 
-/* One CATS decode step in a single kernel launch: everything csffn_gate_mask followed by
- * csffn_sparse_ffn_forward computes, with the same outputs (idx, *count, a_val as gate_mask;
- * out as sparse_ffn_forward).  [CATS] abstract: the gate GEMV, the compare and the flag-gated
- * GEMV of one FFN layer.  One pass over dynamically assigned chunks of neuron rows runs the gate,
- * the threshold, and the up and down projections of the kept rows.  Each CTA adds its partial
- * output into fp32 accumulators in the workspace as soon as its rows are done; after a grid-wide
- * count (cooperative launch) the accumulators become out and are cleared for the next call, and
- * idx / a_val / count are compacted.
- * One launch pays one ramp-up and one tail instead of three.  Runs for 1 <= B <= 4 when
- * d % 128 == 0 (bf16; d % 64 for fp32) and the tokens fit in shared memory beside the weight
- * buffers; other shapes fall back to the two-call path inside this call.  The mask and a_val are
- * bit-for-bit repeatable; out may differ from launch to launch in the last bits (rows reach CTAs
- * dynamically and the CTAs' fp32 partial sums are added in arrival order).  cand_idx / cand_count (both or
- * neither): as in csffn_gate_mask, only the listed neurons (ascending, device count) are
- * considered, e.g. the set csffn_predict_lowrank predicts ([SVDP] Fig. 3: the gate runs on the
- * predicted set; with act = RELU and t = 0 the kept set is {z > 0} within it).  ws sized by
- * csffn_workspace_size for this layer and batch.  B == 0: writes *count = 0. */
+/* One CATS decode step: everything csffn_gate_mask followed by csffn_sparse_ffn_forward computes,
+ * with the same outputs (idx, *count, a_val as gate_mask; out as sparse_ffn_forward).  [CATS]
+ * abstract: the gate GEMV, the compare and the flag-gated GEMV of one FFN layer.  The path depends on
+ * the batch:
+ *   - B <= 2 (and B <= 4 for the shapes the tensor-core path below does not take): a streaming
+ *     kernel runs the gate, the threshold and the up and down projections of the kept rows in one
+ *     pass over dynamically assigned neuron rows, the CTAs adding their partial outputs into fp32
+ *     accumulators in the workspace; a short finishing kernel, launched as its programmatic
+ *     dependent, turns the accumulators into out (clearing them for the next call) and compacts
+ *     idx / a_val / count.  Where that kernel does not fit (d, dtype), a one-launch cooperative
+ *     kernel or the two-call path inside this call computes the same.
+ *   - B >= 3 for bf16 layers with d % 64 == 0 and h % 8 == 0 (no cand_idx): the union of the tokens'
+ *     masks covers most neurons, so the tensor-core FFN of csffn_dense_ffn_forward runs with the
+ *     activations at or below the threshold zeroed, and its down kernel also compacts the keep flags.
+ *   - other shapes: the two-call path inside this call.
+ * The mask and a_val are bit-for-bit repeatable; out may differ from launch to launch in the last
+ * bits on the streaming paths (rows reach CTAs dynamically and the CTAs' fp32 partial sums are added
+ * in arrival order).  cand_idx / cand_count (both or neither): as in csffn_gate_mask, only the
+ * listed neurons (ascending, device count) are considered, e.g. the set csffn_predict_lowrank
+ * predicts ([SVDP] Fig. 3: the gate runs on the predicted set; with act = RELU and t = 0 the kept set
+ * is {z > 0} within it).  ws sized by csffn_workspace_size for this layer and batch.  B == 0: writes
+ * *count = 0. */
 csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int B, float t,
                                     const int32_t* cand_idx, const int32_t* cand_count,
                                     int32_t* idx, int32_t* count, float* a_val,
@@ -180,11 +185,13 @@ csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x
 /* Dense gated FFN over all h neurons (the full model that verifies a chunk of
  * sparse-drafted tokens, [SIRIUS] "Approach"; also the speed-up baseline).
  *   out = (act(x W_gate^T + beta) * (x W_up^T)) W_down.  B == 0: no-op.
- *   bf16 layers with 8 <= B <= 16, d % 128 == 0 and d <= 8192 run on the tensor cores (the
- *   16-token verify chunk: bf16 MMA with fp32 accumulation, one pass over the weights for all
- *   tokens); the down projection takes the fp32 activations as a bf16 high part plus a bf16
- *   low part, so about 16 of their mantissa bits reach the product.  Other calls run on the
- *   CUDA cores (fp32 FMA). */
+ *   bf16 layers with d % 64 == 0 and h % 8 == 0 run on the fifth-generation tensor cores for any
+ *   1 <= B <= 16 (tcgen05 MMA with fp32 accumulators in tensor memory, operands staged by TMA, one
+ *   pass over the weights for all tokens; a gate/up kernel, then a down kernel); the down
+ *   projection takes the fp32 activations as a bf16 high part plus a bf16 low part, so about 16 of
+ *   their mantissa bits reach the product.  The result is bit-for-bit repeatable.  Other bf16 layers
+ *   with 8 <= B <= 16 and d % 128 == 0 use an mma.sync path; the rest runs on the CUDA cores (fp32
+ *   FMA). */
 csffn_status csffn_dense_ffn_forward(const csffn_layer* layer, const void* x, int B,
                                      void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
 
@@ -200,23 +207,36 @@ csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int 
                                    int32_t* cand_idx, int32_t* cand_count,
                                    void* ws, size_t ws_bytes, void* stream);
 
-/* The predictor pipeline of one decode step in a single kernel launch ([SVDP] Fig. 1 and Fig. 3):
- * csffn_predict_lowrank followed by csffn_cats_ffn_forward on the predicted set computes the same.
+/* The predictor pipeline of one decode step ([SVDP] Fig. 1 and Fig. 3): csffn_predict_lowrank
+ * followed by csffn_cats_ffn_forward on the predicted set computes the same.
  *   y = x U_r; neuron i is predicted iff p[b,i] = y_b . V_r[i,:] + beta_i > tau[i] for some token b;
  *   a predicted neuron's gate runs (z = x W_gate[i] + beta_i, a = act(z), token b keeps it iff
  *   |a| > t: with act = RELU and t = 0, A = {z > 0} within the predicted set), and the kept rows'
  *   up and down projections give out.  idx[0 .. *count) = ascending kept neurons, a_val as in
  *   csffn_gate_mask, out as in csffn_sparse_ffn_forward.  The predicted set itself is not written.
  *   u_rt [rank, d], v_r [h, rank] in layer->wdtype, rank % (8 for bf16, 4 for fp32) == 0.
- *   Runs for the shapes csffn_cats_ffn_forward takes in one launch, with a chunk of V_r rows
- *   (at least 8 rows, at most 64 KB where the rank allows) and y beside them in shared memory;
- *   other shapes return CSFFN_ERR_UNSUPPORTED_SHAPE (use the two calls).  The mask and a_val are
- *   bit-for-bit repeatable; out may differ from launch to launch in the last bits, as in
- *   csffn_cats_ffn_forward.  ws sized by csffn_workspace_size(layer, B, rank).  B == 0: writes
- *   *count = 0. */
+ *   1 <= B <= 4: two kernels, y = x U_r, then the rest of the step, chained so that the second
+ *   stages its V_r rows while the first runs (for layers with h <= 256 x the SM count whose V_r rows,
+ *   tokens and a few weight rows fit in shared memory; other shapes take one launch where
+ *   csffn_cats_ffn_forward would).  Other shapes and B > 4 return CSFFN_ERR_UNSUPPORTED_SHAPE (use
+ *   csffn_predict_lowrank, then csffn_cats_ffn_forward on the predicted set).  The
+ *   mask and a_val are bit-for-bit repeatable; out may differ from launch to launch in the last
+ *   bits (the CTAs' partial outputs meet in L2 in arrival order).  ws sized by
+ *   csffn_workspace_size(layer, B, rank).  B == 0: writes *count = 0. */
 csffn_status csffn_svd_ffn_forward(const csffn_layer* layer, const void* x, int B, int rank, const void* u_rt,
                                    const void* v_r, const float* tau, float t, int32_t* idx, int32_t* count,
                                    float* a_val, void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* The same step with the parallel pipeline ([SVDP] Table 3, "Parallel pipeline"; Table 2, "r=1024
+ * parallel"): W_up is read with W_gate for every predicted neuron, so the up projection does not
+ * wait for the gate's decision; the down projection still reads only the kept rows.  The outputs
+ * are those of csffn_svd_ffn_forward (v is zero outside the kept set either way); the difference is
+ * which rows are read.  Runs for the two-kernel shapes above (1 <= B <= 4); other shapes return
+ * CSFFN_ERR_UNSUPPORTED_SHAPE. */
+csffn_status csffn_svd_ffn_forward_parallel(const csffn_layer* layer, const void* x, int B, int rank,
+                                            const void* u_rt, const void* v_r, const float* tau, float t,
+                                            int32_t* idx, int32_t* count, float* a_val, void* out, int out_mode,
+                                            void* ws, size_t ws_bytes, void* stream);
 
 /* Workspace bytes for csffn_calibrate_threshold with n calibration vectors. */
 size_t csffn_calibrate_workspace_size(const csffn_layer* layer, int n, int mode, int rank);

@@ -224,11 +224,16 @@ def test_one_launch_step_empty_candidate_list():
     assert int(cnt.item()) == 0 and torch.all(out == 0)
 
 
-@pytest.mark.parametrize("d,h,r,B", [(1024, 2048, 128, 1), (1024, 2048, 128, 4), (4096, 11008, 256, 1),
-                                     (4096, 11008, 1024, 1), (4096, 11008, 256, 3)])
-def test_one_launch_svd_step(d, h, r, B):
-    """csffn_svd_ffn_forward (predictor, gate on the predicted set, up and down in one launch) against
-    the predictor + one-launch-on-candidates path and the oracle's sequential ReGLU."""
+@pytest.mark.parametrize("d,h,r,B,parallel", [(1024, 2048, 128, 1, False), (1024, 2048, 128, 4, False),
+                                              (4096, 11008, 256, 1, False), (4096, 11008, 1024, 1, False),
+                                              (4096, 11008, 256, 3, False), (1024, 2048, 128, 1, True),
+                                              (1024, 2048, 128, 4, True), (4096, 11008, 256, 1, True),
+                                              (4096, 11008, 1024, 1, True), (4096, 11008, 256, 3, True)])
+def test_one_launch_svd_step(d, h, r, B, parallel):
+    """csffn_svd_ffn_forward (sequential pipeline: y = x U_r, then predictor, gate on the predicted
+    set, up and down on the kept set) and csffn_svd_ffn_forward_parallel
+    (W_up read with W_gate on the predicted set) against the predictor + one-launch-on-candidates
+    path and the oracle's sequential and parallel ReGLU."""
     spec, x, xc, urt, vr, tau_ref = reglu_case(d, h, r, 512)
     x = x[:B]
     layer = dev_layer(spec)
@@ -239,7 +244,7 @@ def test_one_launch_svd_step(d, h, r, B):
     cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
     av = torch.zeros(B, h, device="cuda")
     out = torch.full((B, d), float("nan"), device="cuda")
-    cs.svd_ffn_forward(layer, xd, urt_d, vr_d, tau, 0.0, idx, cnt, av, out, ws)
+    cs.svd_ffn_forward(layer, xd, urt_d, vr_d, tau, 0.0, idx, cnt, av, out, ws, parallel=parallel)
     assert cs.check_status(ws) == 0
     n = int(cnt.item())
     idx1 = idx[:n].cpu().numpy()
@@ -263,6 +268,9 @@ def test_one_launch_svd_step(d, h, r, B):
     amask[:, idx1] = av1 != 0.0
     ref, _ = oracle.reglu_sequential(x, spec, amask)
     assert oracle.rel_l2(out1, ref) <= 1e-4
+    if not _pred_band(p, tau64, rms).any():  # the predicted set is then the oracle's exactly
+        ref_par, a_par = oracle.reglu_parallel(x, spec, np.broadcast_to(pred, (B, h)))
+        assert oracle.rel_l2(out1, ref_par) <= 1e-4  # a gate near zero contributes almost nothing
     # the same step as two calls (predictor, then the one-launch step on its candidates)
     ci = torch.zeros(h, dtype=torch.int32, device="cuda")
     cc = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -275,3 +283,47 @@ def test_one_launch_svd_step(d, h, r, B):
     got2 = np.zeros(h, bool)
     got2[idx2[:int(cnt2.item())].cpu().numpy()] = True
     assert np.array_equal(got[clear], got2[clear])
+
+
+@pytest.mark.parametrize("parallel", [False, True])
+def test_svd_step_whitened_factors(parallel):
+    """Data-whitened factors from the offline stage (contextual_sparsity_ffn_b200.offline, computed on
+    the device from the calibration tokens) through csffn_calibrate_threshold (per-neuron tau) and the
+    SVD step, against the oracle's predictor on the same bf16 factors and its sequential ReGLU."""
+    from contextual_sparsity_ffn_b200 import offline
+    d, h, r, B = 4096, 11008, 256, 1
+    # More calibration vectors than d: with fewer the whitened factors fit the calibration span and
+    # predict almost nothing on other tokens (512 vectors: 0.04% of the neurons on the eval tokens)
+    spec, x, xc = synth.reglu_sparse(0, d=d, h=h, n_eval=4, n_calib=8192)
+    x = x[:B]
+    layer = dev_layer(spec)
+    urt_d, vr_d = offline.svd_predictor_factors(layer.w_gate, r, dev(xc).float())
+    tau = torch.zeros(h, device="cuda")
+    cs.calibrate_threshold(layer, dev(xc), 0.9, _abi.CAL_PER_NEURON_PRED, tau, u_rt=urt_d, v_r=vr_d)
+    urt, vr = cs.to_numpy_bits(urt_d), cs.to_numpy_bits(vr_d)
+    tau64 = tau.cpu().numpy().astype(np.float64)
+    ws = cs.new_workspace(layer, B, r)
+    idx = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    av = torch.zeros(B, h, device="cuda")
+    out = torch.full((B, d), float("nan"), device="cuda")
+    cs.svd_ffn_forward(layer, dev(x), urt_d, vr_d, tau, 0.0, idx, cnt, av, out, ws, parallel=parallel)
+    assert cs.check_status(ws) == 0
+    n = int(cnt.item())
+    idx1 = idx[:n].cpu().numpy()
+    av1 = av[:, :n].cpu().numpy().astype(np.float64)
+    assert_index_list(idx1, h)
+    p = oracle.predict(x, urt, vr, spec.bias)
+    p_cal = oracle.predict(xc[:512], urt, vr, spec.bias)
+    rms = np.sqrt(np.mean(p_cal * p_cal, axis=0))
+    pred = oracle.union_mask(oracle.predicted_mask(p, tau64))
+    z = oracle.gate_preactivation(x, spec)
+    clear = ~_pred_band(p, tau64, rms) & (np.abs(z) > 1e-3 * np.sqrt(np.mean(z * z))).all(axis=0)
+    got = np.zeros(h, bool)
+    got[idx1] = True
+    assert np.array_equal(got[clear], (pred & (z > 0).any(axis=0))[clear])
+    amask = np.zeros((B, h), bool)
+    amask[:, idx1] = av1 != 0.0
+    ref, _ = oracle.reglu_sequential(x, spec, amask)
+    assert oracle.rel_l2(out.cpu().numpy().astype(np.float64), ref) <= 1e-4
+    assert 0.01 < pred.mean() < 0.3  # a predicted set of some hundreds of neurons (about 3.6% here)
