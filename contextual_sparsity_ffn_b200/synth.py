@@ -129,6 +129,17 @@ def reglu_sparse(layer_id: int = 0, d: int = 4096, h: int = 11008, n_eval: int =
     return layer, x, xc
 
 
+def sparse_qwen2_reglu(layer_id: int = 0, n_eval: int = 1, n_calib: int = 512) -> tuple:
+    """Workload 5: ReGLU layer of the SparseQwen2-7B FFN shape (d 3584, h 18944), gate offsets as in
+    workload 2: (layer, eval tokens bf16 unit RMS, calibration tokens)."""
+    d, h = 3584, 18944
+    s = reglu_bias_sigma(d)
+    layer = make_layer(5, layer_id, d, h, "bf16", "relu", bias_mean_std=(-1.5 * s, 0.5 * s))
+    x = make_tokens(5, layer_id, ROLE_EVAL, n_eval, d, "bf16", rms_normalise=True)
+    xc = make_tokens(5, layer_id, ROLE_CALIB, n_calib, d, "bf16", rms_normalise=True)
+    return layer, x, xc
+
+
 def llama3_8b_stack_layer(layer_id: int) -> LayerSpec:
     """Workload 3: one of the 32 LLaMA-3-8B-shaped SwiGLU layers."""
     return make_layer(3, layer_id, 4096, 14336, "bf16", "silu")

@@ -76,10 +76,12 @@ def assert_index_list(idx: np.ndarray, h: int) -> None:
     assert np.all(np.diff(idx) > 0), "indices must be unique and ascending"
 
 
-def check_values(a_val, idx, a_ref, m, t):
+def check_values(a_val, idx, a_ref, m, t, atol_rel=1e-6):
     """a_val against the oracle's activations, element by element: a where the token keeps the row,
-    0 where it rejects it; the per-token masks agree with the oracle's outside the band."""
+    0 where it rejects it; the per-token masks agree with the oracle's outside the band.  atol_rel
+    scales the absolute tolerance by the largest |a| (1e-6 for fp32 sums of one row in order; the
+    tensor-core path adds 64-element partial sums, a few times that)."""
     tb = np.abs(np.abs(a_ref) - t) < 1e-3 * abs(t)
     assert np.array_equal(m[~tb], oracle.cats_mask(a_ref, t)[~tb])
     np.testing.assert_allclose(a_val, np.where(m, a_ref, 0.0)[:, idx], rtol=1e-4,
-                               atol=1e-6 * np.abs(a_ref).max())
+                               atol=atol_rel * np.abs(a_ref).max())
