@@ -26,6 +26,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -217,7 +218,10 @@ def build_workload(torch, cs, synth, sparsities):
 
 
 def run_graph_steps(torch, step_fn, steps, warmup, stream, events_cb=None):
-    """Capture `steps` calls of step_fn(k) into one graph; replay warm-up, then time one replay."""
+    """Capture `steps` calls of step_fn(k) into one graph; replay warm-up, then time one replay.
+    The capture stream first waits for the default stream, where the inputs and workspaces were
+    made (a workspace's counters are zeroed there by csffn_workspace_init)."""
+    stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         for k in range(min(warmup, 3)):
             step_fn(k)
@@ -355,6 +359,14 @@ def sirius_measure(torch, cs, stream, world, dev, rounds=3):
     sparse = torch.zeros(T, d, device=dev)
     dense = torch.zeros(T, d, device=dev)
     t_dev = torch.zeros(1, device=dev)
+    thresholds = {}
+    for s in (0.5, 0.9):
+        thresholds[s] = []
+        for layer in layers:
+            cs.calibrate_threshold(layer, xc, s, cs._abi.CAL_GLOBAL_ABS_ACT, t_dev)
+            thresholds[s].append(float(t_dev.item()))
+        if not all(math.isfinite(t) for t in thresholds[s]):
+            raise RuntimeError(f"calibration gave {thresholds[s]} at s = {s}")
 
     def dense_tokens(k):
         for layer in layers:
@@ -367,10 +379,7 @@ def sirius_measure(torch, cs, stream, world, dev, rounds=3):
     res = {"path": "16 x csffn_cats_ffn_forward (batch 1) + csffn_dense_ffn_forward (batch 16) per layer",
            "dense_16_steps_us_per_layer": round(t_dense * 1e3, 1)}
     for s in (0.5, 0.9):
-        ts = []
-        for layer in layers:
-            cs.calibrate_threshold(layer, xc, s, cs._abi.CAL_GLOBAL_ABS_ACT, t_dev)
-            ts.append(float(t_dev.item()))
+        ts = thresholds[s]
         rec = []
         stack.sirius_round(layers[0], x, ts[0], sparse, dense, buf, ws_dense, record=rec)
         counts = [len(idx) for idx, _ in rec]
