@@ -172,8 +172,10 @@ def _host_ptr(t: torch.Tensor):
 def cats_ffn_forward_host(layer: FFNLayer, x_host: torch.Tensor, t: float, idx: torch.Tensor,
                           count: torch.Tensor, a_val: torch.Tensor, out_host: torch.Tensor, ws: torch.Tensor,
                           stream=None) -> None:
-    """csffn_cats_ffn_forward_host: x_host and out_host are CPU tensors (pinned memory keeps the
-    copies asynchronous); the result is in out_host once the stream has reached this call's copy."""
+    """csffn_cats_ffn_forward_host: x_host and out_host are CPU tensors.  Pinned (page-locked)
+    tensors are read and written by the step itself over the host link; pageable ones are staged
+    through the workspace by copies.  The result is in out_host once the step has completed on the
+    stream, and x_host must stay unchanged until then."""
     B = x_host.shape[0] if x_host.dim() == 2 else 1
     out_mode = _abi.OUT_BF16 if out_host.dtype == torch.bfloat16 else _abi.OUT_F32
     check(load().csffn_cats_ffn_forward_host(layer.ref(), _host_ptr(x_host), B, float(t), _ptr(idx), _ptr(count),

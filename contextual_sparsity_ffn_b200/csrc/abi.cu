@@ -378,6 +378,18 @@ csffn_status csffn_svd_ffn_forward_parallel(const csffn_layer* layer, const void
                      stream);
 }
 
+// The device address of page-locked host memory mapped into the current device's address space
+// (cudaHostAlloc / cudaMallocHost / cudaHostRegister with unified addressing), or nullptr for any
+// other pointer (pageable memory included).
+static void* mapped_host_ptr(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,
                                          int32_t* idx, int32_t* count, float* a_val,
                                          void* out_host, int out_mode, void* ws, size_t ws_bytes, void* stream) {
@@ -397,6 +409,16 @@ csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x
   if ((st = check_cats_step(layer, xd, B, t, idx, a_val, od, ws, ws_bytes)) != CSFFN_OK) return st;
   const size_t xbytes = (size_t)B * layer->d * esize(layer->wdtype);
   const size_t obytes = (size_t)B * layer->d * (out_mode == CSFFN_OUT_BF16 ? 2 : 4);
+  // Mapped page-locked buffers: a kernel stages the tokens into the workspace over the host link and
+  // the step writes out there directly, so the stream holds only kernels (a step may then start
+  // while the previous one ends).
+  void* xm = mapped_host_ptr(x_host);
+  void* om = xm ? mapped_host_ptr(out_host) : nullptr;
+  if (xm && om && aligned16(xm) && aligned16(om)) {
+    if (launch_stage_tokens(xm, xd, xbytes, s) != cudaSuccess) return CSFFN_ERR_CUDA;
+    return csffn_cats_ffn_forward(layer, xd, B, t, nullptr, nullptr, idx, count, a_val, om, out_mode, ws, ws_bytes,
+                                  stream);
+  }
   if (cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return CSFFN_ERR_CUDA;
   st = csffn_cats_ffn_forward(layer, xd, B, t, nullptr, nullptr, idx, count, a_val, od, out_mode, ws, ws_bytes,
                               stream);

@@ -59,7 +59,7 @@ struct WsLayout {
 
 constexpr int kChunkRows = 16;  // rows per compaction chunk (one ballot)
 constexpr int kFusedMaxBatch = 4;
-constexpr int kFusedAccCopies = 4;  // fused step: CTA k adds into accumulator k % kFusedAccCopies
+constexpr int kFusedAccCopies = 8;  // fused step: CTA k adds into accumulator k % kFusedAccCopies
 
 // Tensor-core FFN (tc_ffn.cu): tiles of 128 neurons (gate/up) or 128 output columns (down); at most
 // kTcMaxCtas CTAs, each with two partial-accumulator slots of 32 x 128 floats.

@@ -144,6 +144,9 @@ cudaError_t launch_cats_fused(const FusedArgs& a, int wdtype, cudaStream_t s);
 // bulk copies from one producer warp (ring.cu): one CTA per SM.
 bool cats_ring_supported(int d, int B, int wdtype);
 cudaError_t launch_cats_ring(const FusedArgs& a, int wdtype, cudaStream_t s);
+// Copy of `bytes` (a multiple of 16, both pointers 16-byte aligned) from src (device-accessible, e.g.
+// mapped host memory) to dst, as a programmatic dependent of the kernel before it on the stream.
+cudaError_t launch_stage_tokens(const void* src, void* dst, size_t bytes, cudaStream_t s);
 
 // SVD-predicted step of up to 4 tokens in one cooperative launch (svd_step.cu): y = x U_r, one
 // grid-wide count, then predictor, gate, up, down and the end phase; `parallel` fetches W_up with

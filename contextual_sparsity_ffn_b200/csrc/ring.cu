@@ -333,16 +333,31 @@ __global__ void __launch_bounds__(kRingThreads, 1) cats_ring_kernel(const FusedA
     uint32_t ticket = 0;  // lane 0: a draw in flight
     if (lane == 0 && n_streams < n_chunks) ticket = atomicAdd(p.tickets, 1u);
     bool drawn = n_streams < n_chunks;
-    // tokens -> shared memory as fp32 (zero past B), then a barrier among the gate warps
-    for (int e = tid - kWarp; e < NB * NV; e += kGateWarps * kWarp) {
-      const int b = e / NV, v = e - b * NV;
-      float f[EPV];
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (b < B) raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const WT*>(p.x) + (size_t)b * d + (size_t)v * EPV);
-      unpack(raw, f);
+    // tokens -> shared memory as fp32 (zero past B), then a barrier among the gate warps; the loads
+    // of a batch all go out before the first conversion
+    constexpr int kXLoads = 4;  // 16-byte token loads per thread and batch
+    for (int e0 = tid - kWarp; e0 < NB * NV; e0 += kXLoads * kGateWarps * kWarp) {
+      uint4 raw[kXLoads];
 #pragma unroll
-      for (int hh = 0; hh < XH; ++hh)
-        xs4[((size_t)b * XH + hh) * NV + v] = make_float4(f[4 * hh], f[4 * hh + 1], f[4 * hh + 2], f[4 * hh + 3]);
+      for (int u = 0; u < kXLoads; ++u) {
+        const int e = e0 + u * kGateWarps * kWarp;
+        const int b = e / NV, v = e - b * NV;
+        raw[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (e < NB * NV && b < B)
+          raw[u] = *reinterpret_cast<const uint4*>(reinterpret_cast<const WT*>(p.x) + (size_t)b * d + (size_t)v * EPV);
+      }
+#pragma unroll
+      for (int u = 0; u < kXLoads; ++u) {
+        const int e = e0 + u * kGateWarps * kWarp;
+        if (e < NB * NV) {
+          const int b = e / NV, v = e - b * NV;
+          float f[EPV];
+          unpack(raw[u], f);
+#pragma unroll
+          for (int hh = 0; hh < XH; ++hh)
+            xs4[((size_t)b * XH + hh) * NV + v] = make_float4(f[4 * hh], f[4 * hh + 1], f[4 * hh + 2], f[4 * hh + 3]);
+        }
+      }
     }
     named_sync(1, kGateWarps * kWarp);
 
@@ -662,6 +677,35 @@ static cudaError_t ring_kv_t(const FusedArgs& a, int kv, cudaStream_t s) {
     default: break;
   }
   return cudaErrorInvalidValue;
+}
+
+// Tokens from mapped page-locked host memory into the workspace, once per step, so that the step's
+// CTAs read them from device memory and not each over the host link.  A programmatic dependent of the
+// kernel before it: it copies only after griddepcontrol.wait (the previous step may still read dst,
+// and the source may be an earlier step's output), and the step's kernel after it may start early.
+__global__ void __launch_bounds__(512) stage_tokens_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          int n16) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n16) dst[i] = src[i];
+}
+
+cudaError_t launch_stage_tokens(const void* src, void* dst, size_t bytes, cudaStream_t s) {
+  if (bytes % 16 != 0 || ((uintptr_t)src & 15u) || ((uintptr_t)dst & 15u)) return cudaErrorInvalidValue;
+  const int n16 = (int)(bytes / 16);
+  if (n16 == 0) return cudaSuccess;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n16 + 511) / 512));
+  cfg.blockDim = dim3(512);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, stage_tokens_kernel, reinterpret_cast<const uint4*>(src),
+                            reinterpret_cast<uint4*>(dst), n16);
 }
 
 cudaError_t launch_cats_ring(const FusedArgs& a, int wdtype, cudaStream_t s) {

@@ -171,13 +171,18 @@ csffn_status csffn_cats_ffn_forward(const csffn_layer* layer, const void* x, int
                                     int32_t* idx, int32_t* count, float* a_val,
                                     void* out, int out_mode, void* ws, size_t ws_bytes, void* stream);
 
-/* csffn_cats_ffn_forward with the tokens and the output in host memory: copies x_host [B, d]
- * (weight dtype) into the workspace, runs the one-launch step, and copies out [B, d] (bf16 or fp32;
- * out_mode CSFFN_OUT_BF16 or CSFFN_OUT_F32) back to out_host, all asynchronously on `stream`.
- * idx, count and a_val stay in device memory as in csffn_cats_ffn_forward.  The host buffers must
- * stay valid until the stream reaches the copies; page-locked (pinned) host memory keeps the
- * copies asynchronous, pageable memory makes them synchronous.  ws sized by csffn_workspace_size
- * for this layer and batch (it holds the staged tokens and output).  B == 0: writes *count = 0. */
+/* csffn_cats_ffn_forward with the tokens x_host [B, d] (weight dtype) and the output out_host [B, d]
+ * (bf16 or fp32; out_mode CSFFN_OUT_BF16 or CSFFN_OUT_F32) in host memory, asynchronously on
+ * `stream`.  When both are page-locked host memory mapped into the device's address space
+ * (cudaHostAlloc, cudaMallocHost or cudaHostRegister under unified addressing) and 16-byte aligned,
+ * a small kernel stages x into the workspace over the host link and the step writes out there
+ * directly: no copy-engine work, and consecutive steps on the stream stay chained like
+ * device-memory steps.  Otherwise x is copied into the workspace, the step runs there, and out is
+ * copied back (pageable memory makes those copies synchronous).  idx,
+ * count and a_val stay in device memory as in csffn_cats_ffn_forward.  The host buffers must stay
+ * valid, and x_host unchanged, until the step has completed on the stream.  ws sized by
+ * csffn_workspace_size for this layer and batch (it holds the staged tokens and output).  B == 0:
+ * writes *count = 0. */
 csffn_status csffn_cats_ffn_forward_host(const csffn_layer* layer, const void* x_host, int B, float t,
                                          int32_t* idx, int32_t* count, float* a_val,
                                          void* out_host, int out_mode, void* ws, size_t ws_bytes, void* stream);
