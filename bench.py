@@ -301,9 +301,10 @@ def stack_measure(torch, cs, stream, world, dev, n_steps=4):
     ws16 = cs.new_workspace(layers[0], 16)
     ts = stack.calibrate_stack(layers, h_cal, 0.5, ws16)
     h0 = torch.randn(16, d, generator=gen, device=dev)
-    res = {"path": "per layer csffn_rmsnorm_bf16 + csffn_cats_ffn_forward (accumulate; batch 1 and 4 run as "
-                   "the two-kernel step, batch 16 as the gate mask then the gathered up/down); the dense "
-                   "stack: csffn_rmsnorm_bf16 + csffn_dense_ffn_forward", "layers": L, "target_sparsity": 0.5}
+    res = {"path": "per layer csffn_rmsnorm_bf16 + csffn_cats_ffn_forward (accumulate; batch 1 runs the "
+                   "streaming kernel and its finishing kernel, batch 4 and 16 the tensor-core FFN with the "
+                   "threshold applied); the dense stack: csffn_rmsnorm_bf16 + csffn_dense_ffn_forward",
+           "layers": L, "target_sparsity": 0.5}
     for B in (1, 4, 16):
         sb = stack.stack_buffers(layers[0], B)
         hb = torch.empty(B, d, device=dev)
