@@ -623,16 +623,17 @@ static cudaError_t ring_t(const FusedArgs& a, cudaStream_t st) {
   const RingGeom geo = ring_geom(a.d, (int)sizeof(WT), NB);
   if (geo.lr < 0) return cudaErrorInvalidValue;
   const size_t smem = ring_smem(a.d, (int)sizeof(WT), NB, geo).total;
-  // The shared-memory attribute and the one-CTA-per-SM check, once per device and instance (again
-  // when a larger shape needs more shared memory).
+  // The shared-memory attribute on every call: it belongs to the CUDA context, which a device reset
+  // replaces.  The one-CTA-per-SM check once per device and instance (again when a larger shape
+  // needs more shared memory).
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   static int ready[64] = {0};
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (ready[dev] < (int)smem) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRingThreads, smem);
     if (e != cudaSuccess) return e;
