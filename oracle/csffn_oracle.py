@@ -240,6 +240,34 @@ def calibrate_per_neuron(x_cal, u_rt, v_r, bias, q: float) -> np.ndarray:
     return p[k - 1, :].copy()
 
 
+def recall_thresholds(p: np.ndarray, z: np.ndarray, recall: float) -> np.ndarray:
+    """Per-neuron thresholds that reach a target recall of the truly active set on the calibration
+    vectors ([SVDP] Table 3, "+ Bias calibration", and Fig. 2: with a zero threshold the predictor
+    misses active neurons; the thresholds are moved per neuron to recover them).  The reading: for
+    neuron i, the active calibration vectors are A_i = {n : z_i(x_n) > 0} (m_i of them); c_i =
+    ceil(R * m_i) of them must be predicted, so tau_i is the largest value below the c_i-th largest
+    of {p_i(x_n) : n in A_i}, and p_i > tau_i holds exactly for the predictor outputs at or above
+    it.  tau_i = +inf when c_i = 0 (no active vector, or R = 0): the neuron is never predicted.
+
+    p, z: [N, h]; returns tau [h] in p's precision.
+    """
+    p = np.asarray(p)
+    z = np.asarray(z)
+    tau = np.full(p.shape[1], np.inf, dtype=p.dtype)
+    for i in range(p.shape[1]):
+        act = np.sort(p[z[:, i] > 0, i])
+        c = order_statistic_rank(recall, act.size)
+        if c > 0:
+            tau[i] = np.nextafter(act[act.size - c], -np.inf)
+    return tau
+
+
+def calibrate_per_neuron_recall(x_cal, u_rt, v_r, layer, recall: float) -> np.ndarray:
+    """recall_thresholds on the predictor outputs p = (x U_r) V_r^T + beta and the gate
+    pre-activations z = x W_gate^T + beta of the calibration vectors x_cal [N, d]."""
+    return recall_thresholds(predict(x_cal, u_rt, v_r, layer.bias), gate_preactivation(x_cal, layer), recall)
+
+
 def predicted_mask(p: np.ndarray, tau: np.ndarray) -> np.ndarray:
     """[SVDP] Fig. 1 and Fig. 2: a neuron is predicted active when its predictor output exceeds
     its calibrated threshold, P = {i : p_i > tau_i} per token -> [B, h]."""

@@ -303,6 +303,58 @@ def test_predicted_mask_brute_force():
     assert oracle.predicted_mask(p[1:2], tau).tolist() == [by_hand[1]]
 
 
+def _recall_needed(R: float, m: int) -> int:
+    """Brute force: the fewest of m active vectors whose fraction reaches R (R taken at float32)."""
+    r = Fraction(float(np.float32(R)))
+    return next(c for c in range(m + 1) if m == 0 or Fraction(c, m) >= r) if m else 0
+
+
+def test_recall_thresholds_brute_force():
+    """Per-neuron thresholds for a target recall ([SVDP] Table 3 "+ Bias calibration", Fig. 2),
+    checked by their defining properties on a planted case, not by a retyped formula: among the
+    active vectors (z > 0, strictly) at least the brute-force count c is predicted (p > tau), no
+    larger threshold still predicts c of them, the inactive vectors' outputs do not move tau, and
+    tau = +inf when nothing has to be predicted.  Planted: ties among active outputs, z == 0
+    (inactive), inactive vectors holding the largest outputs, a neuron never active, negative p."""
+    N, h = 9, 6
+    rng = np.random.default_rng(11)
+    p = np.round(rng.standard_normal((N, h)), 1)  # one decimal: ties occur
+    z = rng.standard_normal((N, h))
+    z[:, 3] = -np.abs(z[:, 3])           # neuron 3 never active
+    z[0, :] = 0.0                        # z == 0 is inactive
+    p[0, :] = 50.0                       # ... and holds the largest output
+    p[1, 1] = p[2, 1] = p[4, 1] = 0.7    # ties
+    z[[1, 2, 4], 1] = 1.0
+    z[5, 2] = -1.0
+    p[5, 2] = 40.0                       # an inactive vector with a large output
+    for R in (0.0, 0.25, 0.5, 0.6, 0.75, 0.99, 1.0):
+        tau = oracle.recall_thresholds(p, z, R)
+        assert tau.shape == (h,)
+        for i in range(h):
+            act = [n for n in range(N) if z[n, i] > 0]
+            c = _recall_needed(R, len(act))
+            if c == 0:
+                assert tau[i] == np.inf
+                continue
+            kept = sum(p[n, i] > tau[i] for n in act)
+            assert kept >= c, (R, i, kept, c)
+            above = np.nextafter(tau[i], np.inf)
+            assert sum(p[n, i] > above for n in act) < c, (R, i)
+        # the inactive vectors' outputs do not matter
+        q = p.copy()
+        q[z <= 0] = rng.standard_normal(int((z <= 0).sum())) * 100.0
+        np.testing.assert_array_equal(oracle.recall_thresholds(q, z, R), tau)
+    assert oracle.recall_thresholds(p, z, 1.0)[3] == np.inf
+    # written out by hand: active outputs 0.1, 0.5, 0.5, 0.9 (and an inactive 5.0)
+    pp = np.array([[0.1], [0.5], [0.5], [0.9], [5.0]])
+    zz = np.array([[1.0], [2.0], [0.5], [0.1], [-1.0]])
+    below = lambda v: np.nextafter(v, -np.inf)
+    assert oracle.recall_thresholds(pp, zz, 0.5)[0] == below(0.5)   # c = 2: 0.5, 0.5, 0.9 kept
+    assert oracle.recall_thresholds(pp, zz, 0.75)[0] == below(0.5)  # c = 3
+    assert oracle.recall_thresholds(pp, zz, 1.0)[0] == below(0.1)   # c = 4: all active kept
+    assert oracle.recall_thresholds(pp, zz, 0.25)[0] == below(0.9)  # c = 1
+
+
 # ----------------------------------------------------------------------------- SVD
 
 def test_svd_full_rank_reconstructs_gate():
@@ -453,6 +505,7 @@ PIN_TESTS = [
     lambda: test_reglu_parallel_brute_force(),
     lambda: test_round_effective_density_by_hand(),
     lambda: test_draft_agreement_by_hand(),
+    lambda: test_recall_thresholds_brute_force(),
 ]
 
 
@@ -549,6 +602,46 @@ def _mut_agreement_argmin(sparse_out, dense_out, proj):
             "top1": np.argmin(s @ r, axis=1) == np.argmin(dn @ r, axis=1)}
 
 
+def _mut_recall_all_vectors(p, z, recall):
+    tau = np.full(p.shape[1], np.inf)
+    for i in range(p.shape[1]):
+        act = np.sort(p[:, i])
+        c = oracle.order_statistic_rank(recall, act.size)
+        if c > 0:
+            tau[i] = np.nextafter(act[act.size - c], -np.inf)
+    return tau
+
+
+def _mut_recall_at_value(p, z, recall):
+    tau = np.full(p.shape[1], np.inf)
+    for i in range(p.shape[1]):
+        act = np.sort(p[z[:, i] > 0, i])
+        c = oracle.order_statistic_rank(recall, act.size)
+        if c > 0:
+            tau[i] = act[act.size - c]
+    return tau
+
+
+def _mut_recall_floor(p, z, recall):
+    tau = np.full(p.shape[1], np.inf)
+    for i in range(p.shape[1]):
+        act = np.sort(p[z[:, i] > 0, i])
+        c = math.floor(float(np.float32(recall)) * act.size)
+        if c > 0:
+            tau[i] = np.nextafter(act[act.size - c], -np.inf)
+    return tau
+
+
+def _mut_recall_zero_active(p, z, recall):
+    tau = np.full(p.shape[1], np.inf)
+    for i in range(p.shape[1]):
+        act = np.sort(p[z[:, i] >= 0, i])
+        c = oracle.order_statistic_rank(recall, act.size)
+        if c > 0:
+            tau[i] = np.nextafter(act[act.size - c], -np.inf)
+    return tau
+
+
 MUTANTS = {
     "silu_sign": ("silu", _mut_silu_sign),
     "dropped_bias": ("gate_preactivation", _mut_no_bias),
@@ -567,6 +660,10 @@ MUTANTS = {
     "parallel_no_relu": ("reglu_parallel", _mut_parallel_no_relu),
     "density_no_verify": ("round_effective_density", _mut_density_no_verify),
     "agreement_argmin": ("draft_agreement", _mut_agreement_argmin),
+    "recall_all_vectors": ("recall_thresholds", _mut_recall_all_vectors),
+    "recall_at_value": ("recall_thresholds", _mut_recall_at_value),
+    "recall_floor": ("recall_thresholds", _mut_recall_floor),
+    "recall_zero_active": ("recall_thresholds", _mut_recall_zero_active),
 }
 
 
