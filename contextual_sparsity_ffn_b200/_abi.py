@@ -17,7 +17,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CU
 BF16, F32 = 0, 1
 OUT_BF16, OUT_F32, OUT_F32_ACCUMULATE = 0, 1, 2
 ACT_SILU, ACT_RELU = 0, 1
-CAL_GLOBAL_ABS_ACT, CAL_PER_NEURON_PRED = 0, 1
+CAL_GLOBAL_ABS_ACT, CAL_PER_NEURON_PRED, CAL_PER_NEURON_RECALL = 0, 1, 2
 MAX_BATCH = 16
 
 

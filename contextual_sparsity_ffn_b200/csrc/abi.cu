@@ -566,23 +566,29 @@ csffn_status csffn_predict_lowrank(const csffn_layer* layer, const void* x, int 
 namespace {
 constexpr size_t kHeaderBytes = 512;
 struct CalLayout {
-  size_t kth, values, y, total;
+  size_t kth, values, y, zt, total;
 };
 CalLayout cal_layout(const csffn_layer* L, int n, int mode, int rank) {
   CalLayout c;
+  const bool pred = mode == CSFFN_CAL_PER_NEURON_PRED || mode == CSFFN_CAL_PER_NEURON_RECALL;
   size_t o = kHeaderBytes;
   c.kth = o;    o += kth_state_bytes();
   c.values = o; o += align_up(sizeof(float) * (size_t)n * L->h, 256);
-  c.y = o;      o += mode == CSFFN_CAL_PER_NEURON_PRED ? align_up(sizeof(float) * (size_t)n * rank, 256) : 0;
+  c.y = o;      o += pred ? align_up(sizeof(float) * (size_t)n * rank, 256) : 0;
+  c.zt = o;     o += mode == CSFFN_CAL_PER_NEURON_RECALL ? align_up(sizeof(float) * (size_t)n * L->h, 256) : 0;
   c.total = o;
   return c;
+}
+
+bool cal_mode_ok(int mode) {
+  return mode == CSFFN_CAL_GLOBAL_ABS_ACT || mode == CSFFN_CAL_PER_NEURON_PRED || mode == CSFFN_CAL_PER_NEURON_RECALL;
 }
 }  // namespace
 
 size_t csffn_calibrate_workspace_size(const csffn_layer* layer, int n, int mode, int rank) {
   if (check_layer_shape(layer) != CSFFN_OK || n < 1 || n > CSFFN_MAX_CALIB) return 0;
-  if (mode != CSFFN_CAL_GLOBAL_ABS_ACT && mode != CSFFN_CAL_PER_NEURON_PRED) return 0;
-  if (mode == CSFFN_CAL_PER_NEURON_PRED && (rank < 1 || rank > CSFFN_MAX_RANK)) return 0;
+  if (!cal_mode_ok(mode)) return 0;
+  if (mode != CSFFN_CAL_GLOBAL_ABS_ACT && (rank < 1 || rank > CSFFN_MAX_RANK)) return 0;
   return cal_layout(layer, n, mode, rank).total;
 }
 
@@ -594,7 +600,7 @@ csffn_status csffn_calibrate_threshold(const csffn_layer* layer, const void* x_c
   if (st != CSFFN_OK) return st;
   if (!x_cal || !t_out || n < 1 || n > CSFFN_MAX_CALIB) return CSFFN_ERR_INVALID_ARG;
   if (!(target_sparsity >= 0.f && target_sparsity <= 1.f)) return CSFFN_ERR_INVALID_ARG;
-  if (mode != CSFFN_CAL_GLOBAL_ABS_ACT && mode != CSFFN_CAL_PER_NEURON_PRED) return CSFFN_ERR_INVALID_ARG;
+  if (!cal_mode_ok(mode)) return CSFFN_ERR_INVALID_ARG;
   if (!aligned16(x_cal)) return CSFFN_ERR_ALIGNMENT;
   const int group_cap = CSFFN_MAX_BATCH;
   int group = group_cap;
@@ -627,15 +633,17 @@ csffn_status csffn_calibrate_threshold(const csffn_layer* layer, const void* x_c
     return cuda_status(launch_kth_smallest(vals, M, k, t_out, at<void>(ws, C.kth), s));
   }
 
-  // PER_NEURON_PRED
+  // PER_NEURON_PRED and PER_NEURON_RECALL
+  const bool recall = mode == CSFFN_CAL_PER_NEURON_RECALL;
   if (!u_rt || !v_r) return CSFFN_ERR_INVALID_ARG;
   if (rank < 1 || rank > CSFFN_MAX_RANK) return CSFFN_ERR_INVALID_ARG;
   if (rank % vec_elems(layer->wdtype) != 0) return CSFFN_ERR_ALIGNMENT;
   if (!aligned16(u_rt) || !aligned16(v_r)) return CSFFN_ERR_ALIGNMENT;
+  if (recall && (st = check_weights(layer, true, false, false)) != CSFFN_OK) return st;
   const CalLayout C = cal_layout(layer, n, mode, rank);
   if ((st = check_ws(ws, ws_bytes, C.total)) != CSFFN_OK) return st;
   const long long k = exact_rank(target_sparsity, n);
-  if (k == 0) return cuda_status(launch_fill(t_out, -INFINITY, layer->h, s));
+  if (!recall && k == 0) return cuda_status(launch_fill(t_out, -INFINITY, layer->h, s));
   float* y = at<float>(ws, C.y);
   float* pt = at<float>(ws, C.values);  // P^T [h][n]
   int pgroup = group;
@@ -666,7 +674,23 @@ csffn_status csffn_calibrate_threshold(const csffn_layer* layer, const void* x_c
     g.transpose_out = 1;
     if (launch_row_gemv(g, layer->wdtype, layer->wdtype == CSFFN_BF16, s) != cudaSuccess) return CSFFN_ERR_CUDA;
   }
-  return cuda_status(launch_rows_kth(pt, layer->h, n, (int)k, t_out, s));
+  if (!recall) return cuda_status(launch_rows_kth(pt, layer->h, n, (int)k, t_out, s));
+  float* zt = at<float>(ws, C.zt);  // Z^T [h][n]: the gate pre-activations
+  for (int b0 = 0; b0 < n; b0 += group) {
+    RowGemvArgs g{};
+    g.W = layer->w_gate;
+    g.x = reinterpret_cast<const char*>(x_cal) + (size_t)b0 * xrow;
+    g.rows = layer->h;
+    g.K = layer->d;
+    g.B = (n - b0) < group ? (n - b0) : group;
+    g.y = zt + b0;
+    g.y_stride = n;
+    g.bias = layer->gate_bias;
+    g.act = -1;
+    g.transpose_out = 1;
+    if (launch_row_gemv(g, layer->wdtype, false, s) != cudaSuccess) return CSFFN_ERR_CUDA;
+  }
+  return cuda_status(launch_rows_recall(pt, zt, layer->h, n, target_sparsity, t_out, s));
 }
 
 size_t csffn_kth_workspace_size(void) { return kHeaderBytes + kth_state_bytes(); }

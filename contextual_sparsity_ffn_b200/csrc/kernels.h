@@ -191,6 +191,9 @@ size_t kth_state_bytes();
 cudaError_t launch_kth_smallest(const float* values, int64_t n, int64_t k, float* out, void* state,
                                 cudaStream_t s);
 cudaError_t launch_rows_kth(const float* values, int rows, int n, int k, float* out, cudaStream_t s);
+// Per-neuron thresholds for a target recall of the active set (rows of P^T and Z^T, n vectors each).
+cudaError_t launch_rows_recall(const float* pt, const float* zt, int rows, int n, float recall, float* out,
+                               cudaStream_t s);
 cudaError_t launch_fill(float* p, float v, int n, cudaStream_t s);
 
 cudaError_t launch_rmsnorm_bf16(const float* h, int B, int d, float eps, void* xn, cudaStream_t s);

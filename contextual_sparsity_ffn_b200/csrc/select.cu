@@ -97,14 +97,9 @@ cudaError_t launch_kth_smallest(const float* values, int64_t n, int64_t k, float
   return cudaGetLastError();
 }
 
-// out[r] = k-th smallest (1-indexed) of values[r*n .. r*n + n), by a bitonic sort in shared
-// memory (n padded with +inf up to a power of two).
-__global__ void __launch_bounds__(256) rows_kth_kernel(const float* __restrict__ values, int n, int n2,
-                                                       int k, float* __restrict__ out) {
-  extern __shared__ float sv[];
-  const float* row = values + (size_t)blockIdx.x * n;
-  for (int i = threadIdx.x; i < n2; i += blockDim.x) sv[i] = i < n ? row[i] : __int_as_float(0x7f800000);
-  __syncthreads();
+// Ascending bitonic sort of sv[0, n2) in shared memory by the whole block (n2 a power of two); the
+// block's threads are synchronised on return.
+__device__ void block_bitonic_sort(float* sv, int n2) {
   for (int kk = 2; kk <= n2; kk <<= 1) {
     for (int j = kk >> 1; j > 0; j >>= 1) {
       for (int i = threadIdx.x; i < n2; i += blockDim.x) {
@@ -121,6 +116,17 @@ __global__ void __launch_bounds__(256) rows_kth_kernel(const float* __restrict__
       __syncthreads();
     }
   }
+}
+
+// out[r] = k-th smallest (1-indexed) of values[r*n .. r*n + n), by a bitonic sort in shared
+// memory (n padded with +inf up to a power of two).
+__global__ void __launch_bounds__(256) rows_kth_kernel(const float* __restrict__ values, int n, int n2,
+                                                       int k, float* __restrict__ out) {
+  extern __shared__ float sv[];
+  const float* row = values + (size_t)blockIdx.x * n;
+  for (int i = threadIdx.x; i < n2; i += blockDim.x) sv[i] = i < n ? row[i] : __int_as_float(0x7f800000);
+  __syncthreads();
+  block_bitonic_sort(sv, n2);
   if (threadIdx.x == 0) out[blockIdx.x] = sv[k - 1];
 }
 
@@ -133,6 +139,61 @@ cudaError_t launch_rows_kth(const float* values, int rows, int n, int k, float* 
     if (e != cudaSuccess) return e;
   }
   rows_kth_kernel<<<rows, 256, smem, s>>>(values, n, n2, k, out);
+  return cudaGetLastError();
+}
+
+// ceil(R * m) for a float R in [0, 1] and 0 <= m < 2^31, exactly: R = mant * 2^-sh with a 24-bit
+// integer mant, so R * m = mant * m / 2^sh with the numerator below 2^55.
+__device__ __forceinline__ int exact_ceil_mul(float R, int m) {
+  if (!(R > 0.f) || m <= 0) return 0;
+  const uint32_t b = __float_as_uint(R);
+  const int e = (int)((b >> 23) & 0xffu);
+  const unsigned long long mant = e ? ((b & 0x7fffffu) | 0x800000u) : (b & 0x7fffffu);
+  const int sh = e ? 150 - e : 149;
+  const unsigned long long num = mant * (unsigned long long)m;
+  unsigned long long q = sh >= 64 ? (num ? 1ull : 0ull) : ((num >> sh) + (((num >> sh) << sh) != num ? 1ull : 0ull));
+  return q > (unsigned long long)m ? m : (int)q;
+}
+
+// Per-neuron thresholds for a target recall R of the active set: row r of pt and zt holds the
+// predictor outputs p_r and the gate pre-activations z_r of the n calibration vectors.  The outputs
+// of the active vectors (z > 0) are sorted, the others set to +inf; with m active and c = ceil(R m),
+// out[r] is the largest float below the c-th largest active output (so p > out[r] holds for exactly
+// the outputs at or above it), or +inf when c = 0.
+__global__ void __launch_bounds__(256) rows_recall_kernel(const float* __restrict__ pt, const float* __restrict__ zt,
+                                                          int n, int n2, float R, float* __restrict__ out) {
+  extern __shared__ float sv[];
+  __shared__ int s_m;
+  const float* prow = pt + (size_t)blockIdx.x * n;
+  const float* zrow = zt + (size_t)blockIdx.x * n;
+  if (threadIdx.x == 0) s_m = 0;
+  __syncthreads();
+  int m = 0;
+  for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+    const bool active = i < n && zrow[i] > 0.f;
+    sv[i] = active ? prow[i] : __int_as_float(0x7f800000);
+    m += active ? 1 : 0;
+  }
+  atomicAdd(&s_m, m);
+  __syncthreads();
+  block_bitonic_sort(sv, n2);
+  if (threadIdx.x == 0) {
+    const int ma = s_m;
+    const int c = exact_ceil_mul(R, ma);
+    out[blockIdx.x] = c == 0 ? __int_as_float(0x7f800000) : nextafterf(sv[ma - c], -INFINITY);
+  }
+}
+
+cudaError_t launch_rows_recall(const float* pt, const float* zt, int rows, int n, float recall, float* out,
+                               cudaStream_t s) {
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  const size_t smem = (size_t)n2 * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(rows_recall_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  rows_recall_kernel<<<rows, 256, smem, s>>>(pt, zt, n, n2, recall, out);
   return cudaGetLastError();
 }
 

@@ -82,7 +82,8 @@ typedef enum { CSFFN_ACT_SILU = 0, CSFFN_ACT_RELU = 1 } csffn_act;
 
 typedef enum {
   CSFFN_CAL_GLOBAL_ABS_ACT = 0,  /* one scalar t: quantile of |a| over calibration set x neurons [CATS] */
-  CSFFN_CAL_PER_NEURON_PRED = 1  /* tau[h]: per-neuron quantile of the SVD predictor output [SVDP] Fig. 1 */
+  CSFFN_CAL_PER_NEURON_PRED = 1, /* tau[h]: per-neuron quantile of the SVD predictor output [SVDP] Fig. 1 */
+  CSFFN_CAL_PER_NEURON_RECALL = 2 /* tau[h]: per-neuron target recall of {z > 0} [SVDP] Table 3, Fig. 2 */
 } csffn_cal_mode;
 
 /* One gated FFN layer.  wdtype applies to w_gate, w_up, w_down_t and to x. */
@@ -254,6 +255,11 @@ size_t csffn_calibrate_workspace_size(const csffn_layer* layer, int n, int mode,
  *   PER_NEURON_PRED: p as in csffn_predict_lowrank for each calibration vector;
  *     k = ceil(s*n); t_out[i] = k-th smallest of {p_i(x_n)} (t_out is [h]), or
  *     -inf when k == 0.
+ *   PER_NEURON_RECALL: s is the target recall R.  p as above and z = x.W_gate[i] + beta_i for
+ *     each calibration vector; with A_i = {n : z_i(x_n) > 0}, m_i = |A_i| and c_i = ceil(R*m_i)
+ *     (exact), t_out[i] = the largest float below the c_i-th largest of {p_i(x_n) : n in A_i}, so
+ *     that p_i > t_out[i] predicts at least c_i of them; +inf when c_i == 0 (never predicted).
+ *     Needs w_gate (and gate_bias when the layer has one).
  *   1 <= n <= CSFFN_MAX_CALIB, 0 <= s <= 1. */
 csffn_status csffn_calibrate_threshold(const csffn_layer* layer, const void* x_cal, int n,
                                        float target_sparsity, int mode,

@@ -128,6 +128,18 @@ def test_calibrate_validation(lib):
     assert lib.csffn_calibrate_workspace_size(ctypes.byref(L), 512, 0, 0) >= 512 * 11008 * 4
     assert lib.csffn_calibrate_workspace_size(ctypes.byref(L), 512, 1, 0) == 0
     assert lib.csffn_calibrate_workspace_size(ctypes.byref(L), 0, 0, 0) == 0
+    # the recall mode: the predictor's factors, aligned, and the gate weights (it needs z too)
+    assert c(mode=_abi.CAL_PER_NEURON_RECALL, rank=256, u=0) == _abi.ERR_INVALID_ARG
+    assert c(mode=_abi.CAL_PER_NEURON_RECALL, rank=100, u=FAKE) == _abi.ERR_ALIGNMENT
+    no_gate = layer()
+    no_gate.w_gate = None
+    assert f(ctypes.byref(no_gate), P(FAKE), 512, 0.9, _abi.CAL_PER_NEURON_RECALL, P(FAKE), P(FAKE), 256, P(FAKE),
+             P(FAKE), BIG, None) == _abi.ERR_INVALID_ARG
+    assert c(mode=_abi.CAL_PER_NEURON_RECALL, rank=256, u=FAKE, s=1.5) == _abi.ERR_INVALID_ARG
+    assert lib.csffn_calibrate_workspace_size(ctypes.byref(L), 512, _abi.CAL_PER_NEURON_RECALL, 0) == 0
+    ws_pred = lib.csffn_calibrate_workspace_size(ctypes.byref(L), 512, _abi.CAL_PER_NEURON_PRED, 256)
+    ws_recall = lib.csffn_calibrate_workspace_size(ctypes.byref(L), 512, _abi.CAL_PER_NEURON_RECALL, 256)
+    assert ws_recall - ws_pred >= 512 * 11008 * 4  # room for z of every calibration vector
 
 
 def test_kth_rmsnorm_selftest_validation(lib):

@@ -102,6 +102,59 @@ def test_per_neuron_calibration(d, h, r):
     np.testing.assert_allclose(tau.cpu().numpy(), tau_ref, rtol=1e-4, atol=1e-5 * rms.max())
 
 
+@pytest.mark.parametrize("d,h,r,n", [(1024, 2048, 128, 512), (4096, 11008, 256, 512), (1024, 1000, 64, 100)])
+@pytest.mark.parametrize("R", [0.0, 0.8, 0.95, 1.0])
+def test_per_neuron_recall_calibration(d, h, r, n, R):
+    """CSFFN_CAL_PER_NEURON_RECALL against oracle.recall_thresholds on the same calibration
+    vectors: tau per neuron (+inf where nothing has to be predicted), wherever the active set is
+    unambiguous (no vector with z within rounding of 0); and the recall the GPU's thresholds reach
+    on the oracle's p and z.  n = 100 is not a power of two (the sort pads it)."""
+    spec, x, xc, urt, vr, _ = reglu_case(d, h, r, n)
+    layer = dev_layer(spec)
+    tau = torch.zeros(h, device="cuda")
+    cs.calibrate_threshold(layer, dev(xc), R, _abi.CAL_PER_NEURON_RECALL, tau, u_rt=dev(urt), v_r=dev(vr))
+    got = tau.cpu().numpy().astype(np.float64)
+    p = oracle.predict(xc, urt, vr, spec.bias)
+    z = oracle.gate_preactivation(xc, spec)
+    ref = oracle.recall_thresholds(p, z, R)
+    zrms = np.sqrt(np.mean(z * z))
+    clear = ~(np.abs(z) < 1e-4 * zrms).any(axis=0)
+    assert clear.mean() > 0.5
+    inf_ref = np.isinf(ref)
+    assert np.array_equal(np.isinf(got)[clear], inf_ref[clear])
+    if R == 0.0:
+        assert np.all(np.isposinf(got))
+        return
+    fin = clear & ~inf_ref
+    assert fin.any()
+    prms = np.sqrt(np.mean(p * p, axis=0))
+    np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-4, atol=1e-5 * prms.max())
+    # the recall reached on the calibration set by every neuron with a clear active set: at least
+    # c_i = ceil(R m_i) of its m_i active vectors predicted.  Each threshold sits just below one
+    # vector's output, which the fp32 and fp64 sums may put on either side of it, so a vector within
+    # rounding of tau counts as predicted.
+    act = (z > 0)[:, clear]
+    tol = 1e-5 * prms.max()
+    hit = (p[:, clear] > got[clear][None, :] - tol) & act
+    need = np.array([oracle.order_statistic_rank(R, int(m)) for m in act.sum(axis=0)])
+    assert (hit.sum(axis=0) >= need).all()
+    assert hit.sum() >= R * act.sum()
+    # the thresholds (+inf included) drive the predictor as any others: its candidate list on four
+    # other tokens against the oracle's predicted set, outside the rounding band
+    ws = cs.new_workspace(layer, 4, r)
+    cand_idx = torch.full((h,), -1, dtype=torch.int32, device="cuda")
+    cand_count = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cs.predict_lowrank(layer, dev(x), dev(urt), dev(vr), tau, cand_idx, cand_count, ws)
+    assert cs.check_status(ws) == 0
+    P = cand_idx[:int(cand_count.item())].cpu().numpy()
+    assert_index_list(P, h)
+    pe = oracle.predict(x, urt, vr, spec.bias)
+    band = _pred_band(pe, np.where(np.isinf(got), 0.0, got), prms) & ~np.isinf(got)
+    pm = np.zeros(h, bool)
+    pm[P] = True
+    assert np.array_equal(pm[~band], oracle.union_mask(oracle.predicted_mask(pe, got))[~band])
+
+
 @pytest.mark.parametrize("d,h,r", [(1024, 2048, 128), (4096, 11008, 256), (4096, 11008, 1024)])
 @pytest.mark.parametrize("B", [1, 4])
 def test_predict_gate_reglu_sequential(d, h, r, B):
