@@ -133,6 +133,44 @@ def test_whitened_predictor_beats_naive_on_anisotropic_tokens(capsys):
                                          f"AUROC {v['auroc']:.3f} rel.err {v['rel_err']:.3f}" for k, v in res.items()))
 
 
+def test_recall_targeted_thresholds_on_anisotropic_tokens(capsys):
+    """Per-neuron thresholds set for a target recall R of the truly active set (the pages' Table 3
+    "+ Bias calibration" and Fig. 2, in the reading of oracle.recall_thresholds) on the workload
+    above: set on the 2048 calibration tokens, scored on 2048 others.  The recall carries over to
+    the held-out tokens, a higher R costs predicted density, and the data-whitened factors reach the
+    same recall at a lower density than the naive ones."""
+    d, h = 256, 688
+    layer = synth.make_layer(34, 0, d, h, "f32", "relu")
+    xc, xe = _aniso_tokens(2048, d, seed=1), _aniso_tokens(2048, d, seed=2)
+    zc, ze = oracle.gate_preactivation(xc, layer), oracle.gate_preactivation(xe, layer)
+    active = ze > 0
+    w = _torch_operand(layer.w_gate)
+    rows = []
+    for r in (32, 64):
+        res = {}
+        for name, xcal in (("naive", None), ("whitened", torch.from_numpy(xc))):
+            u_rt, v_r = offline.svd_predictor_factors(w, r, xcal, out_dtype=torch.float64)
+            u_rt, v_r = u_rt.numpy(), v_r.numpy()
+            pc, pe = oracle.predict(xc, u_rt, v_r), oracle.predict(xe, u_rt, v_r)
+            for R in (0.9, 0.95, 0.99):
+                tau = oracle.recall_thresholds(pc, zc, R)
+                cal = (pc > tau[None, :]) & (zc > 0)
+                assert cal.sum() >= R * (zc > 0).sum()  # reached on the calibration set
+                pred = pe > tau[None, :]
+                res[(name, R)] = dict(recall=(pred & active).sum() / active.sum(), density=pred.mean())
+        rows.append((r, res))
+        for R in (0.9, 0.95, 0.99):
+            n, wt = res[("naive", R)], res[("whitened", R)]
+            assert n["recall"] > R - 0.02 and wt["recall"] > R - 0.02
+            assert wt["density"] < n["density"] - 0.01
+        for name in ("naive", "whitened"):
+            assert res[(name, 0.9)]["density"] < res[(name, 0.95)]["density"] < res[(name, 0.99)]["density"]
+    with capsys.disabled():
+        for r, res in rows:
+            print(f"\nr={r}: " + "; ".join(f"{k[0]} R={k[1]}: recall {v['recall']:.3f} density {v['density']:.3f}"
+                                          for k, v in res.items()))
+
+
 def test_artefacts_round_trip_bit_for_bit(tmp_path):
     layer = synth.make_layer(35, 0, 32, 48, "bf16", "relu")
     u_rt, v_r = offline.svd_predictor_factors(_torch_operand(layer.w_gate), 8)
