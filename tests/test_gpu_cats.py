@@ -370,26 +370,28 @@ def test_fused_decode_7b_low_threshold_keeps_negative_activations():
 
 
 @pytest.mark.parametrize("pinned", [True, False])
-def test_fused_decode_host_buffers(pinned):
+@pytest.mark.parametrize("B", [2, 4])
+def test_fused_decode_host_buffers(pinned, B):
     """csffn_cats_ffn_forward_host: tokens in and output out through host memory -- pinned (the step
     reads and writes the mapped host buffers itself) and pageable (staged through the workspace by
     copies) -- checked against the oracle on the call's own mask, and against the device entry
-    point's result (bf16 and fp32 outputs)."""
-    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=2, n_calib=64)
+    point's result (bf16 and fp32 outputs).  B = 2 runs the streaming step, B = 4 the tensor-core
+    FFN in masked mode."""
+    spec, x, xc = synth.llama2_7b_swiglu(0, n_eval=B, n_calib=64)
     t = oracle.calibrate_global(xc, spec, 0.5)
     layer = dev_layer(spec)
-    ws = cs.new_workspace(layer, 2)
+    ws = cs.new_workspace(layer, B)
     idx_d, a_val_d, out_d = run_fused(layer, x, t, ws=ws)
     xh = dev(x).cpu()
     if pinned:
         xh = xh.pin_memory()
     for dtype, tol in ((torch.float32, 1e-6), (torch.bfloat16, TOL_BF16)):
-        oh = torch.full((2, spec.d), float("nan"), dtype=dtype)
+        oh = torch.full((B, spec.d), float("nan"), dtype=dtype)
         if pinned:
             oh = oh.pin_memory()
         idx = torch.zeros(spec.h, dtype=torch.int32, device="cuda")
         cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
-        av = torch.zeros(2, spec.h, device="cuda")
+        av = torch.zeros(B, spec.h, device="cuda")
         cs.cats_ffn_forward_host(layer, xh, t, idx, cnt, av, oh, ws)
         torch.cuda.synchronize()
         assert cs.check_status(ws) == 0
