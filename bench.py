@@ -732,8 +732,8 @@ def time_step_eager(torch, cs, layers, thr, xs, buf, out_t, stream, K):
 def e2e_measure(torch, cs, layers, thr, xs, buf, stream, K, W, world, dev):
     """Same step through the public C-ABI call that takes host buffers (csffn_cats_ffn_forward_host):
     every step takes its token from pinned host memory and puts its output into pinned host memory
-    inside the timed region (the step's kernels read and write the mapped host buffers over the host
-    link); the host waits for all K results at the end."""
+    inside the timed region (the step's kernels read x and write out over the host link: a staging
+    kernel copies x into the workspace once); the host waits for all K results at the end."""
     host_x = xs.cpu().pin_memory()
     host_out = torch.empty(K, D, dtype=torch.float32).pin_memory()
 
@@ -758,9 +758,9 @@ def e2e_measure(torch, cs, layers, thr, xs, buf, stream, K, W, world, dev):
     wall_ms = max_over_ranks(wall_ms, world, dev)
     return {"value": round(whole_job_us_per_layer(wall_ms, K, world), 3), "unit": UNIT,
             "h2d_bytes_per_step": 2 * D, "d2h_bytes_per_step": 4 * D,
-            "how": "csffn_cats_ffn_forward_host, one C-ABI call per step on pinned host buffers (the "
-                   "step reads x from and writes out to mapped host memory over the host link); host "
-                   "wall clock around K steps"}
+            "how": "csffn_cats_ffn_forward_host, one C-ABI call per step on pinned host buffers (a "
+                   "staging kernel reads x over the host link into the workspace, the step writes out "
+                   "into the mapped host buffer); host wall clock around K steps"}
 
 
 # ---------------------------------------------------------------------------------- oracle legs
