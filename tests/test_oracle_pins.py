@@ -180,6 +180,57 @@ def test_cats_sparse_brute_force(d, h):
     np.testing.assert_allclose(out, bf_dense_ffn(x, layer, mask=np.abs(a) > t), rtol=1e-12, atol=1e-15)
 
 
+def test_sparse_ffn_arbitrary_masks_brute_force():
+    """The masked FFN on masks that no threshold produces (a random per-token mask, as the GPU tests
+    pass back in from the kernels' own index lists), a one-row mask broadcast over the tokens, and
+    the empty and full masks, against the per-element loops."""
+    d, h = 12, 20
+    layer = _tiny_layer(d, h)
+    x = _tiny_tokens(3, d)
+    rng = np.random.default_rng(21)
+    m = rng.random((3, h)) < 0.4
+    np.testing.assert_allclose(oracle.sparse_ffn(x, layer, m), bf_dense_ffn(x, layer, mask=m), rtol=1e-12,
+                               atol=1e-15)
+    row = rng.random(h) < 0.5
+    np.testing.assert_allclose(oracle.sparse_ffn(x, layer, row), bf_dense_ffn(x, layer, mask=row), rtol=1e-12,
+                               atol=1e-15)
+    assert np.all(oracle.sparse_ffn(x, layer, np.zeros(h, bool)) == 0.0)
+    np.testing.assert_allclose(oracle.sparse_ffn(x, layer, np.ones((3, h), bool)), bf_dense_ffn(x, layer),
+                               rtol=1e-12, atol=1e-15)
+
+
+def test_recall_calibration_of_a_layer_brute_force():
+    """calibrate_per_neuron_recall on a tiny ReGLU layer with its own factors: the predictor outputs
+    and gate pre-activations recomputed by per-element loops, then the recall property on them (at
+    least ceil(R m_i) of neuron i's active calibration vectors predicted, and no larger threshold
+    predicting as many; +inf where none is needed)."""
+    d, h, r, N = 10, 7, 3, 15
+    s = synth.reglu_bias_sigma(d)
+    layer = _tiny_layer(d, h, act="relu", bias=(-0.5 * s, 0.5 * s))
+    xc = _tiny_tokens(N, d, role=synth.ROLE_CALIB)
+    urt, vr = oracle.svd_factors(layer.w_gate, r)
+    X, Wg, U, V = _f64(xc), _f64(layer.w_gate), np.asarray(urt), np.asarray(vr)
+    beta = _f64(layer.bias)
+    p = np.zeros((N, h))
+    z = np.zeros((N, h))
+    for n in range(N):
+        y = [sum(float(X[n, j]) * float(U[k, j]) for j in range(d)) for k in range(r)]
+        for i in range(h):
+            p[n, i] = sum(y[k] * float(V[i, k]) for k in range(r)) + float(beta[i])
+            z[n, i] = sum(float(X[n, j]) * float(Wg[i, j]) for j in range(d)) + float(beta[i])
+    for R in (0.0, 0.5, 0.9, 1.0):
+        tau = oracle.calibrate_per_neuron_recall(xc, urt, vr, layer, R)
+        for i in range(h):
+            act = [n for n in range(N) if z[n, i] > 0]
+            c = _recall_needed(R, len(act))
+            if c == 0:
+                assert tau[i] == np.inf
+                continue
+            margin = 1e-9 * (1.0 + abs(tau[i]))  # the loops and the library sum in different orders
+            assert sum(p[n, i] > tau[i] - margin for n in act) >= c
+            assert sum(p[n, i] > tau[i] + margin for n in act) < c
+
+
 def test_reglu_sequential_brute_force():
     d, h = 24, 30
     s = synth.reglu_bias_sigma(d)
@@ -506,6 +557,8 @@ PIN_TESTS = [
     lambda: test_round_effective_density_by_hand(),
     lambda: test_draft_agreement_by_hand(),
     lambda: test_recall_thresholds_brute_force(),
+    lambda: test_sparse_ffn_arbitrary_masks_brute_force(),
+    lambda: test_recall_calibration_of_a_layer_brute_force(),
 ]
 
 
